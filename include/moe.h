@@ -1,0 +1,163 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE FFN forward library (libmoe.so).
+ *
+ * One call computes the FFN half of a DeepSeek-V3.2-style MoE transformer block:
+ *
+ *     x, residual = ffn_norm(x, residual)        RMSNorm with the residual add fused in
+ *     out         = ffn(x)                       routed SwiGLU experts + shared expert
+ *
+ * as defined on the DeepSeek-V3.2-Exp model-atlas pages:
+ *   - "MoE update" page, Block excerpt: x, residual = self.ffn_norm(x, residual); x = self.ffn(x).
+ *   - "MoE update" page, RMSNorm.forward excerpt: s = x.float() + residual.float();
+ *     var = mean(s^2); s * rsqrt(var + eps); weight * s; normed and residual cast to x's dtype.
+ *   - "MoE update" / "Add shared output" pages, MoE.forward excerpt and the equation
+ *     delta_ffn = y_routed + y_shared: router weights and indices; every routed (token, slot)
+ *     adds expert(x) * weight into a float32 y; the shared expert is added to every token; y is
+ *     cast to x's dtype with shape [B, T, d].
+ *   - "Gate projection" page: expert = w2((silu(w1 x).float() * (w3 x).float()).type_as(x)),
+ *     weights held [out, in] without bias; 1-byte weights carry one float32 scale per 128x128
+ *     block, scale shape [ceil(out/128), ceil(in/128)].
+ *
+ * The router's body is not on the pages.  This library computes scores = sigmoid(xn . Wg_e +
+ * bias_e) in float32, keeps the top_k experts (on equal scores the lower expert index wins),
+ * normalises their scores to sum 1, and re-decides in float64 every token whose k-th and
+ * (k+1)-th float32 scores are closer than tie_tau.
+ *
+ * Conventions for every entry point
+ *   - Tensors are device pointers (CUDA global memory of the current device), contiguous and
+ *     row-major, 16-byte aligned.  The caller owns all memory; the library allocates none and
+ *     keeps no pointer after a call returns.
+ *   - bf16 = IEEE bfloat16 bits (uint16); e4m3 = OCP FP8 E4M3 codes (uint8).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  Work is
+ *     enqueued on it; moe_forward never synchronises the host.
+ *   - Argument errors are returned synchronously and enqueue nothing.  Launch failures return
+ *     MOE_ERR_CUDA.  Errors found on the device (a bounded wait that gave up) are latched into
+ *     the workspace status word; moe_get_status() reads it.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,     /* NULL pointer, bad size, misaligned pointer, k > E, ... */
+    MOE_ERR_UNSUPPORTED = 2,     /* valid per the pages but not built (see moe_config_t) */
+    MOE_ERR_WORKSPACE = 3,       /* workspace NULL or smaller than moe_workspace_bytes() */
+    MOE_ERR_CUDA = 4,            /* a CUDA runtime/driver call or a launch failed */
+    MOE_ERR_DEVICE_TIMEOUT = 5,  /* a kernel's bounded wait gave up (latched on the device) */
+    MOE_ERR_DEVICE_CHECK = 6     /* a device-side consistency check failed (latched) */
+} moe_status_t;
+
+/* Weight storage ("Gate projection" page, Linear excerpt). */
+typedef enum {
+    MOE_W_BF16 = 0,              /* bf16 [out, in], no scale */
+    MOE_W_FP8_E4M3_B128 = 1      /* e4m3 [out, in] + float32 scale [out/128, in/128] */
+} moe_wtype_t;
+
+/* Precision of the activations fed to the expert GEMMs (the FP8 GEMM body is not on the
+ * pages).  MOE_ACT_FP8_1x128: per token and per 128-column group, sc = amax/448,
+ * q = e4m3(v/sc) -- applied to the normed input and to the SwiGLU hidden state h.
+ * MOE_ACT_BF16: bf16 activations (the only mode for bf16 weights). */
+typedef enum {
+    MOE_ACT_FP8_1x128 = 0,
+    MOE_ACT_BF16 = 1
+} moe_amode_t;
+
+typedef struct {
+    int32_t num_tokens;    /* T = B * S, >= 1 */
+    int32_t dim;           /* d, multiple of 256 */
+    int32_t inter_dim;     /* I (moe_inter_dim), multiple of 128 */
+    int32_t n_experts;     /* E routed experts, 1..256, multiple of 8 or E <= 8 */
+    int32_t top_k;         /* k, 1..E */
+    int32_t shared_inter;  /* width of the shared SwiGLU (n_shared * per-expert inter; several
+                              shared experts are one SwiGLU with concatenated hidden units);
+                              multiple of 128; 0 = no shared expert */
+    int32_t wtype;         /* moe_wtype_t, same for routed and shared weights */
+    int32_t amode;         /* moe_amode_t; FP8 weights need MOE_ACT_FP8_1x128 in this build */
+    float eps;             /* RMSNorm eps (1e-6 on the pages) */
+    float tie_tau;         /* float32 score margin below which a token is re-routed in float64;
+                              <= 0 selects the default 1e-4 */
+} moe_config_t;
+
+/* Expert weights, [out, in] row-major.  Routed: w1, w3 [E, I, d]; w2 [E, d, I].
+ * Scales (FP8 only, else NULL): s1, s3 [E, I/128, d/128]; s2 [E, d/128, I/128].
+ * Shared (NULL when shared_inter == 0): sw1, sw3 [Is, d]; sw2 [d, Is]; ss1, ss3 [Is/128, d/128];
+ * ss2 [d/128, Is/128]. */
+typedef struct {
+    const void *w1, *w3, *w2;
+    const float *s1, *s3, *s2;
+    const void *sw1, *sw3, *sw2;
+    const float *ss1, *ss3, *ss2;
+} moe_weights_t;
+
+/* Bytes of device workspace moe_forward needs for this configuration (0 if cfg is invalid).
+ * The workspace holds every intermediate (normed and quantised activations, logits, routing,
+ * permuted rows, hidden states, expert outputs) and the device status word. */
+size_t moe_workspace_bytes(const moe_config_t* cfg);
+
+/* The fused forward pass.
+ *   x            [T, d] bf16            input of ffn_norm (the attention output)
+ *   residual     [T, d] bf16 or NULL    residual stream; NULL = RMSNorm without the add
+ *   norm_w       [d] float32            RMSNorm gain
+ *   gate_w       [E, d] bf16            router weight
+ *   gate_bias    [E] float32 or NULL    per-expert bias added to the logits before the sigmoid
+ *   w            expert weights (moe_weights_t)
+ *   out          [T, d] bf16            delta_ffn
+ *   residual_out [T, d] bf16            new residual = bf16(x + residual); may equal residual
+ *                                       (in place); unused when residual is NULL
+ *   workspace    >= moe_workspace_bytes(cfg) bytes of device memory, 256-byte aligned; it must
+ *                not be used by another call still running on the device.
+ * No other aliasing is allowed. */
+moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* residual,
+                         const float* norm_w, const void* gate_w, const float* gate_bias,
+                         const moe_weights_t* w, void* out, void* residual_out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* moe_forward that also records caller-created CUDA events (cudaEvent_t passed as void*) on
+ * `stream` at the stage boundaries, for timing individual kernels inside a running workload:
+ *   events[0] before the first launch      events[4] after the permutation kernels
+ *   events[1] after the norm kernel        events[5] after the grouped GEMM up (w1|w3, SwiGLU)
+ *   events[2] after the gate GEMM          events[6] after the grouped GEMM down (w2)
+ *   events[3] after top-k + recheck        events[7] after the combine kernel
+ * n_events may be smaller than 8 (the later boundaries are then not recorded); NULL entries are
+ * skipped.  Same arguments, errors and ownership as moe_forward otherwise. */
+moe_status_t moe_forward_traced(const moe_config_t* cfg, const void* x, const void* residual,
+                                const float* norm_w, const void* gate_w, const float* gate_bias,
+                                const moe_weights_t* w, void* out, void* residual_out,
+                                void* workspace, size_t workspace_bytes, void* stream,
+                                void* const* events, int32_t n_events);
+
+/* Synchronises `stream`, then returns the status latched in the workspace by the last
+ * moe_forward on it (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_CHECK), or MOE_ERR_CUDA. */
+moe_status_t moe_get_status(const void* workspace, void* stream);
+
+/* Copies (device to device, enqueued on `stream`) the routing of the last moe_forward that
+ * used this workspace: idx [T, k] int32 (slot order = descending score), weights [T, k]
+ * float32, counts [E] int32 (tokens per expert), near_tie [T] uint8 (1 = the token was
+ * re-decided in float64).  Any output pointer may be NULL. */
+moe_status_t moe_debug_routing(const moe_config_t* cfg, const void* workspace, int32_t* idx,
+                               float* weights, int32_t* counts, uint8_t* near_tie, void* stream);
+
+/* Copies the normed activations of the last moe_forward: xn [T, d] bf16, and in FP8
+ * activation mode xq [T, d] e4m3 and xs [d/128, T] float32 (group scales, transposed).
+ * Any output pointer may be NULL. */
+moe_status_t moe_debug_norm(const moe_config_t* cfg, const void* workspace, void* xn,
+                            void* xq, float* xs, void* stream);
+
+/* Number of kernel launches one moe_forward enqueues for this configuration. */
+int32_t moe_launches_per_forward(const moe_config_t* cfg);
+
+/* Static description of a status code. */
+const char* moe_status_string(moe_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

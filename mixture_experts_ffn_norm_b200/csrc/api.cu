@@ -1,0 +1,393 @@
+// Host side of libmoe: argument checks, workspace layout, TMA tensor maps and the launch
+// sequence of one forward pass.  Nothing here waits on the device except moe_get_status.
+//
+// Launch sequence (one stream, no host sync; every routing-dependent size is read on the device):
+//   norm -> gate GEMM (logits) -> top-k -> float64 near-tie recheck -> hist -> scan -> scatter
+//   -> gather -> grouped GEMM up (w1|w3 + SwiGLU) -> grouped GEMM down (w2) -> combine
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+}  // namespace
+
+int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// 2-D map over a row-major [rows, inner] tensor of 1-byte (fp8) or 2-byte (bf16) elements; box =
+// 128 bytes x 128 rows, 128-byte swizzle, out-of-range rows read as zero.
+bool encode_map_2d(CUtensorMap* map, const void* base, bool fp8, uint64_t inner, uint64_t rows) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * (fp8 ? 1u : 2u)};
+    const cuuint32_t box[2] = {fp8 ? 128u : 64u, 128u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_layout(const moe_config_t& c, Layout& L) {
+    if (c.num_tokens < 1 || c.dim < 256 || c.dim % 256 || c.inter_dim < 128 || c.inter_dim % 128) return false;
+    if (c.n_experts < 1 || c.n_experts > kMaxExperts || (c.n_experts > 8 && c.n_experts % 8)) return false;
+    if (c.top_k < 1 || c.top_k > c.n_experts) return false;
+    if (c.shared_inter < 0 || c.shared_inter % 128) return false;
+    if (c.wtype != MOE_W_BF16 && c.wtype != MOE_W_FP8_E4M3_B128) return false;
+    if (c.amode != MOE_ACT_FP8_1x128 && c.amode != MOE_ACT_BF16) return false;
+    if (!(c.eps >= 0.0f)) return false;
+    if (static_cast<long long>(c.num_tokens) * c.top_k > (1ll << 30)) return false;
+    L.T = c.num_tokens;
+    L.d = c.dim;
+    L.I = c.inter_dim;
+    L.E = c.n_experts;
+    L.k = c.top_k;
+    L.Is = c.shared_inter;
+    L.fp8 = c.wtype == MOE_W_FP8_E4M3_B128;
+    L.act8 = L.fp8;
+    L.Tpad = static_cast<int>(align_up(L.T, kBM));
+    L.R = static_cast<int>(align_up(static_cast<size_t>(L.T) * L.k + static_cast<size_t>(L.E) * (kBM - 1), kBM));
+    L.KBd = L.d / 128;
+    L.KBi = L.I / 128;
+    L.KBs = L.Is / 128;
+    L.nchunks = (L.T * L.k + kRouteChunk - 1) / kRouteChunk;
+    const size_t ab = L.act8 ? 1 : 2;   // bytes per activation element fed to the expert GEMMs
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align_up(o + bytes, 1024);
+        return at;
+    };
+    L.status = take(kStatusWords * 4);
+    L.xn = take(static_cast<size_t>(L.T) * L.d * 2);
+    L.xq = take(L.act8 ? static_cast<size_t>(L.T) * L.d : 0);
+    L.xs = take(L.act8 ? static_cast<size_t>(L.KBd) * L.Tpad * 4 : 0);
+    L.logits = take(static_cast<size_t>(L.T) * L.E * 4);
+    L.idx = take(static_cast<size_t>(L.T) * L.k * 4);
+    L.w = take(static_cast<size_t>(L.T) * L.k * 4);
+    L.flag = take(L.T);
+    L.flag_list = take(static_cast<size_t>(L.T) * 4);
+    L.counts = take(static_cast<size_t>(L.E) * 4);
+    L.offsets = take(static_cast<size_t>(L.E + 1) * 4);
+    L.row_base = take(static_cast<size_t>(L.E + 1) * 4);
+    L.row_count = take(static_cast<size_t>(L.E + 1) * 4);
+    L.ts_up = take(static_cast<size_t>(L.E + 2) * 4);
+    L.ts_down = take(static_cast<size_t>(L.E + 2) * 4);
+    L.chunk_hist = take(static_cast<size_t>(L.nchunks) * L.E * 4);
+    L.row_of = take(static_cast<size_t>(L.T) * L.k * 4);
+    L.row_token = take(static_cast<size_t>(L.R) * 4);
+    L.a_perm = take(static_cast<size_t>(L.R) * L.d * ab);
+    L.as_perm = take(L.act8 ? static_cast<size_t>(L.KBd) * L.R * 4 : 0);
+    L.h = take(static_cast<size_t>(L.R) * L.I * ab);
+    L.hs = take(L.act8 ? static_cast<size_t>(L.KBi) * L.R * 4 : 0);
+    L.h_sh = take(static_cast<size_t>(L.Tpad) * L.Is * ab);
+    L.hs_sh = take(L.act8 ? static_cast<size_t>(L.KBs) * L.Tpad * 4 : 0);
+    L.y = take(static_cast<size_t>(L.R) * L.d * 2);
+    L.y_sh = take(static_cast<size_t>(L.T) * L.d * 2);
+    L.total = o;
+    return true;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+moe_status_t check_config(const moe_config_t* cfg, Layout& L) {
+    if (!cfg || !make_layout(*cfg, L)) return MOE_ERR_INVALID_ARG;
+    if (cfg->wtype == MOE_W_BF16 && cfg->amode != MOE_ACT_BF16) return MOE_ERR_INVALID_ARG;
+    if (cfg->wtype == MOE_W_FP8_E4M3_B128 && cfg->amode != MOE_ACT_FP8_1x128) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+#define MOE_TRY(expr)                          \
+    do {                                       \
+        if ((expr) != cudaSuccess) return MOE_ERR_CUDA; \
+    } while (0)
+
+}  // namespace
+
+extern "C" size_t moe_workspace_bytes(const moe_config_t* cfg) {
+    Layout L;
+    if (check_config(cfg, L) != MOE_OK) return 0;
+    return L.total;
+}
+
+extern "C" int32_t moe_launches_per_forward(const moe_config_t* cfg) {
+    Layout L;
+    if (check_config(cfg, L) != MOE_OK) return 0;
+    return 11;   // norm, gate GEMM, top-k, recheck, hist, scan, scatter, gather, up, down, combine
+}
+
+static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const void* residual,
+                                 const float* norm_w, const void* gate_w, const float* gate_bias,
+                                 const moe_weights_t* w, void* out, void* residual_out, void* workspace,
+                                 size_t workspace_bytes, void* stream_, void* const* events, int n_events) {
+    Layout L;
+    moe_status_t st = check_config(cfg, L);
+    if (st != MOE_OK) return st;
+    if (!x || !norm_w || !gate_w || !w || !out) return MOE_ERR_INVALID_ARG;
+    if (residual && !residual_out) return MOE_ERR_INVALID_ARG;
+    if (!w->w1 || !w->w3 || !w->w2) return MOE_ERR_INVALID_ARG;
+    if (L.fp8 && (!w->s1 || !w->s3 || !w->s2)) return MOE_ERR_INVALID_ARG;
+    if (L.Is > 0) {
+        if (!w->sw1 || !w->sw3 || !w->sw2) return MOE_ERR_INVALID_ARG;
+        if (L.fp8 && (!w->ss1 || !w->ss3 || !w->ss2)) return MOE_ERR_INVALID_ARG;
+    }
+    const void* ptrs[] = {x, residual, norm_w, gate_w, gate_bias, w->w1, w->w3, w->w2, w->sw1, w->sw3, w->sw2,
+                          out, residual_out};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return MOE_ERR_WORKSPACE;
+    if (out == x || out == residual || (residual_out && (residual_out == x || residual_out == out)))
+        return MOE_ERR_INVALID_ARG;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream_);
+    auto mark = [&](int i) {
+        return (events && i < n_events && events[i]) ? cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s)
+                                                     : cudaSuccess;
+    };
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const float tau = cfg->tie_tau > 0.0f ? cfg->tie_tau : 1e-4f;
+    const int sms = num_sms();
+    const bool fp8 = L.fp8;
+
+    MOE_TRY(cudaMemsetAsync(ws + L.status, 0, kStatusWords * 4, s));
+    MOE_TRY(cudaMemsetAsync(ws + L.row_token, 0xFF, static_cast<size_t>(L.R) * 4, s));
+    MOE_TRY(mark(0));
+
+    // 1. ffn_norm (+ FP8 activation quant)
+    MOE_TRY(launch_norm(L, x, residual, norm_w, cfg->eps, residual_out, ws, s));
+    MOE_TRY(mark(1));
+
+    // 2. router logits on the tensor cores: xn [T, d] x Wg [E, d]^T
+    {
+        TensorMaps m;
+        if (!encode_map_2d(&m.a_s, ws + L.xn, false, L.d, L.T) || !encode_map_2d(&m.b0_s, gate_w, false, L.d, L.E))
+            return MOE_ERR_CUDA;
+        m.a_r = m.a_s;
+        m.b1_s = m.b0_s;
+        m.b0_r = m.b0_s;
+        m.b1_r = m.b0_s;
+        GemmParams p{};
+        p.G = 1;
+        p.single_rows = L.T;
+        p.n_tiles_s = 1;
+        p.kb_s = L.d / 64;
+        p.out_s = ws + L.logits;
+        p.out_ld_s = L.E;
+        p.n_valid_cols = L.E;
+        p.status = reinterpret_cast<uint32_t*>(ws + L.status);
+        const int tiles = (L.T + kBM - 1) / kBM;
+        MOE_TRY(launch_gemm(kModeLogits, false, m, p, std::min(tiles, sms), s));
+    }
+    MOE_TRY(mark(2));
+    // 3. top-k + float64 recheck of near ties
+    MOE_TRY(launch_topk(L, gate_bias, tau, ws, s));
+    MOE_TRY(launch_recheck(L, gate_w, gate_bias, ws, s));
+    MOE_TRY(mark(3));
+
+    // 4. permutation by expert
+    const int ntu_r = L.I / 128, ntu_s = L.Is / 128, ntd = L.d / 256;
+    MOE_TRY(launch_route(L, ntu_r, ntu_s, ntd, ntd, ws, s));
+    MOE_TRY(mark(4));
+
+    const int G = L.E + (L.Is > 0 ? 1 : 0);
+    const int max_tiles_up = (L.R / kBM) * ntu_r + (L.Is > 0 ? (L.Tpad / kBM) * ntu_s : 0);
+    const int max_tiles_down = (L.R / kBM) * ntd + (L.Is > 0 ? (L.Tpad / kBM) * ntd : 0);
+
+    // 5. grouped GEMM up: h = silu(a W1^T) * (a W3^T)
+    {
+        TensorMaps m;
+        bool ok = encode_map_2d(&m.a_r, ws + L.a_perm, fp8, L.d, L.R) &&
+                  encode_map_2d(&m.a_s, ws + (fp8 ? L.xq : L.xn), fp8, L.d, L.T) &&
+                  encode_map_2d(&m.b0_r, w->w1, fp8, L.d, static_cast<uint64_t>(L.E) * L.I) &&
+                  encode_map_2d(&m.b1_r, w->w3, fp8, L.d, static_cast<uint64_t>(L.E) * L.I);
+        if (L.Is > 0)
+            ok = ok && encode_map_2d(&m.b0_s, w->sw1, fp8, L.d, L.Is) && encode_map_2d(&m.b1_s, w->sw3, fp8, L.d, L.Is);
+        else
+            m.b0_s = m.b0_r, m.b1_s = m.b1_r;
+        if (!ok) return MOE_ERR_CUDA;
+        GemmParams p{};
+        p.G = G;
+        p.has_shared = L.Is > 0;
+        p.tile_start = reinterpret_cast<const int*>(ws + L.ts_up);
+        p.row_base = reinterpret_cast<const int*>(ws + L.row_base);
+        p.row_count = reinterpret_cast<const int*>(ws + L.row_count);
+        p.n_tiles_r = ntu_r;
+        p.n_tiles_s = ntu_s;
+        p.kb_r = p.kb_s = fp8 ? L.d / 128 : L.d / 64;
+        p.b_rows_per_expert = L.I;
+        p.as_r = reinterpret_cast<const float*>(ws + L.as_perm);
+        p.as_s = reinterpret_cast<const float*>(ws + L.xs);
+        p.as_ld_r = L.R;
+        p.as_ld_s = L.Tpad;
+        p.bs0_r = w->s1;
+        p.bs1_r = w->s3;
+        p.bs0_s = w->ss1;
+        p.bs1_s = w->ss3;
+        p.bs_cols_r = p.bs_cols_s = L.d / 128;
+        p.bs_rows_r = L.I / 128;
+        p.out_r = ws + L.h;
+        p.out_s = ws + L.h_sh;
+        p.out_ld_r = L.I;
+        p.out_ld_s = L.Is;
+        p.outs_r = reinterpret_cast<float*>(ws + L.hs);
+        p.outs_s = reinterpret_cast<float*>(ws + L.hs_sh);
+        p.outs_ld_r = L.R;
+        p.outs_ld_s = L.Tpad;
+        p.status = reinterpret_cast<uint32_t*>(ws + L.status);
+        MOE_TRY(launch_gemm(kModeUp, fp8, m, p, std::min(max_tiles_up, sms), s));
+    }
+    MOE_TRY(mark(5));
+    // 6. grouped GEMM down: y = h W2^T
+    {
+        TensorMaps m;
+        bool ok = encode_map_2d(&m.a_r, ws + L.h, fp8, L.I, L.R) &&
+                  encode_map_2d(&m.b0_r, w->w2, fp8, L.I, static_cast<uint64_t>(L.E) * L.d);
+        m.b1_r = m.b0_r;
+        if (L.Is > 0) {
+            ok = ok && encode_map_2d(&m.a_s, ws + L.h_sh, fp8, L.Is, L.Tpad) &&
+                 encode_map_2d(&m.b0_s, w->sw2, fp8, L.Is, L.d);
+            m.b1_s = m.b0_s;
+        } else {
+            m.a_s = m.a_r, m.b0_s = m.b0_r, m.b1_s = m.b0_r;
+        }
+        if (!ok) return MOE_ERR_CUDA;
+        GemmParams p{};
+        p.G = G;
+        p.has_shared = L.Is > 0;
+        p.tile_start = reinterpret_cast<const int*>(ws + L.ts_down);
+        p.row_base = reinterpret_cast<const int*>(ws + L.row_base);
+        p.row_count = reinterpret_cast<const int*>(ws + L.row_count);
+        p.n_tiles_r = p.n_tiles_s = ntd;
+        p.kb_r = fp8 ? L.I / 128 : L.I / 64;
+        p.kb_s = fp8 ? L.Is / 128 : L.Is / 64;
+        p.b_rows_per_expert = L.d;
+        p.as_r = reinterpret_cast<const float*>(ws + L.hs);
+        p.as_s = reinterpret_cast<const float*>(ws + L.hs_sh);
+        p.as_ld_r = L.R;
+        p.as_ld_s = L.Tpad;
+        p.bs0_r = p.bs1_r = w->s2;
+        p.bs0_s = p.bs1_s = w->ss2;
+        p.bs_cols_r = L.I / 128;
+        p.bs_cols_s = L.Is / 128;
+        p.bs_rows_r = L.d / 128;
+        p.out_r = ws + L.y;
+        p.out_s = ws + L.y_sh;
+        p.out_ld_r = p.out_ld_s = L.d;
+        p.status = reinterpret_cast<uint32_t*>(ws + L.status);
+        MOE_TRY(launch_gemm(kModeDown, fp8, m, p, std::min(max_tiles_down, sms), s));
+    }
+    MOE_TRY(mark(6));
+    // 7. weighted combine + shared add -> out
+    MOE_TRY(launch_combine(L, out, ws, s));
+    MOE_TRY(mark(7));
+    return MOE_OK;
+}
+
+extern "C" moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* residual,
+                                    const float* norm_w, const void* gate_w, const float* gate_bias,
+                                    const moe_weights_t* w, void* out, void* residual_out, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+    return forward_impl(cfg, x, residual, norm_w, gate_w, gate_bias, w, out, residual_out, workspace,
+                        workspace_bytes, stream, nullptr, 0);
+}
+
+extern "C" moe_status_t moe_forward_traced(const moe_config_t* cfg, const void* x, const void* residual,
+                                           const float* norm_w, const void* gate_w, const float* gate_bias,
+                                           const moe_weights_t* w, void* out, void* residual_out, void* workspace,
+                                           size_t workspace_bytes, void* stream, void* const* events,
+                                           int32_t n_events) {
+    return forward_impl(cfg, x, residual, norm_w, gate_w, gate_bias, w, out, residual_out, workspace,
+                        workspace_bytes, stream, events, n_events);
+}
+
+extern "C" moe_status_t moe_get_status(const void* workspace, void* stream) {
+    if (!workspace) return MOE_ERR_INVALID_ARG;
+    uint32_t st[2] = {0, 0};
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpy(st, workspace, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (st[0] == kErrTimeout) return MOE_ERR_DEVICE_TIMEOUT;
+    if (st[0] != 0) return MOE_ERR_DEVICE_CHECK;
+    return MOE_OK;
+}
+
+extern "C" moe_status_t moe_debug_routing(const moe_config_t* cfg, const void* workspace, int32_t* idx,
+                                          float* weights, int32_t* counts, uint8_t* near_tie, void* stream) {
+    Layout L;
+    moe_status_t st = check_config(cfg, L);
+    if (st != MOE_OK) return st;
+    if (!workspace) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+    const size_t tk = static_cast<size_t>(L.T) * L.k;
+    if (idx) MOE_TRY(cudaMemcpyAsync(idx, ws + L.idx, tk * 4, cudaMemcpyDeviceToDevice, s));
+    if (weights) MOE_TRY(cudaMemcpyAsync(weights, ws + L.w, tk * 4, cudaMemcpyDeviceToDevice, s));
+    if (counts) MOE_TRY(cudaMemcpyAsync(counts, ws + L.counts, static_cast<size_t>(L.E) * 4, cudaMemcpyDeviceToDevice, s));
+    if (near_tie) MOE_TRY(cudaMemcpyAsync(near_tie, ws + L.flag, L.T, cudaMemcpyDeviceToDevice, s));
+    return MOE_OK;
+}
+
+extern "C" moe_status_t moe_debug_norm(const moe_config_t* cfg, const void* workspace, void* xn, void* xq,
+                                       float* xs, void* stream) {
+    Layout L;
+    moe_status_t st = check_config(cfg, L);
+    if (st != MOE_OK) return st;
+    if (!workspace) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+    const size_t td = static_cast<size_t>(L.T) * L.d;
+    if (xn) MOE_TRY(cudaMemcpyAsync(xn, ws + L.xn, td * 2, cudaMemcpyDeviceToDevice, s));
+    if ((xq || xs) && !L.act8) return MOE_ERR_INVALID_ARG;
+    if (xq) MOE_TRY(cudaMemcpyAsync(xq, ws + L.xq, td, cudaMemcpyDeviceToDevice, s));
+    if (xs)
+        MOE_TRY(cudaMemcpy2DAsync(xs, static_cast<size_t>(L.T) * 4, ws + L.xs, static_cast<size_t>(L.Tpad) * 4,
+                                  static_cast<size_t>(L.T) * 4, L.KBd, cudaMemcpyDeviceToDevice, s));
+    return MOE_OK;
+}
+
+extern "C" const char* moe_status_string(moe_status_t s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+        case MOE_ERR_CUDA: return "CUDA call or kernel launch failed";
+        case MOE_ERR_DEVICE_TIMEOUT: return "a device-side bounded wait gave up";
+        case MOE_ERR_DEVICE_CHECK: return "a device-side check failed";
+    }
+    return "unknown status";
+}

@@ -1,0 +1,440 @@
+// Persistent grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM), fed by TMA.
+//
+// One kernel serves the three contractions of the layer:
+//   kModeLogits : router logits  = xn [T, d] . Wg[E, d]^T                 (bf16, one group)
+//   kModeUp     : SwiGLU up      g = a . W1_e^T, u = a . W3_e^T, h = silu(g) * u
+//                 ("Gate projection" page, expert excerpt); w1 and w3 rows share one A tile:
+//                 the B tile is [128 rows of W1 ; 128 rows of W3] and one 128x256 MMA covers both
+//   kModeDown   : SwiGLU down    y = h . W2_e^T
+// over groups = routed experts (rows permuted by expert) + the shared expert (all tokens).
+//
+// FP8 weights carry one float32 scale per 128x128 block ("Gate projection" page, Linear excerpt)
+// and the activations one per 1x128 group, neither a power of two, so the tensor core's own block
+// scaling does not apply.  Each 128-wide K block is therefore accumulated into its own TMEM buffer
+// and promoted by the epilogue warps: acc += P_kb * (s_act[row, kb] * s_w[nblk, kb]) in float32
+// registers.  Two TMEM buffers (2 x 256 columns) let the MMA of block kb+1 run while block kb is
+// promoted.  bf16 operands simply accumulate the whole K in TMEM.
+//
+// Warp roles (320 threads, one CTA per SM, persistent over a device-side tile table):
+//   warp 0      one thread issues the TMA loads of A (128 x 128 B) and B (256 x 128 B) per stage
+//   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=32 bytes per instruction)
+//   warps 2..9  epilogue: warp w reads TMEM lanes 32*(w%4).., column half (w-2)/4
+// Tiles are taken m-fastest inside a group so concurrently running CTAs share the weight tile
+// through L2.  Every wait is bounded (see ptx.cuh); on a timeout all roles leave their loops,
+// in-flight TMA loads and MMAs are drained with bounded waits, and TMEM is freed.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kStageBytes = kStageBytesA + kStageBytesB;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+constexpr uint32_t kTmemCols = 512;
+
+struct Tile {
+    int g, mt, nt, shared, a_row0, rows_valid, kb, b_row0;
+};
+
+__device__ __forceinline__ void decode_tile(int t, const int* ts, const int* rb, const int* rc, const GemmParams& p,
+                                            int mode, Tile& ti) {
+    int lo = 0, hi = p.G;   // largest g with ts[g] <= t (groups without tiles are skipped)
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (ts[mid] <= t) lo = mid;
+        else hi = mid;
+    }
+    ti.g = lo;
+    ti.shared = (p.single_rows > 0) || (p.has_shared && lo == p.G - 1);
+    const int cnt = rc[lo];
+    const int mtiles = (cnt + kBM - 1) / kBM;
+    const int local = t - ts[lo];
+    ti.nt = local / mtiles;
+    ti.mt = local - ti.nt * mtiles;
+    ti.a_row0 = rb[lo] + ti.mt * kBM;
+    ti.rows_valid = min(kBM, cnt - ti.mt * kBM);
+    ti.kb = ti.shared ? p.kb_s : p.kb_r;
+    const int nrows = (mode == kModeUp) ? 128 : 256;
+    ti.b_row0 = (ti.shared ? 0 : lo * p.b_rows_per_expert) + ti.nt * nrows;
+}
+
+// bounded wait without the abort check, for draining copies / MMAs already in flight
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(smem_u32(bar), parity))
+        if (clock64() - t0 > kWaitCycles) return;
+}
+
+__device__ __forceinline__ float bf16r(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(a))) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(b))) << 16);
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+    // silu(g) * u with the Linear outputs g, u in bf16 and the product rounded to bf16
+    const float gb = bf16r(g), ub = bf16r(u);
+    return bf16r((gb / (1.0f + expf(-gb))) * ub);
+}
+
+template <bool kFp8, int kMode>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ CUtensorMap tm_a_s,
+            const __grid_constant__ CUtensorMap tm_b0_r, const __grid_constant__ CUtensorMap tm_b1_r,
+            const __grid_constant__ CUtensorMap tm_b0_s, const __grid_constant__ CUtensorMap tm_b1_s,
+            const GemmParams p) {
+    extern __shared__ uint8_t dyn_smem[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t full_bar[kStages];
+    __shared__ __align__(8) uint64_t empty_bar[kStages];
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ volatile int abort_sh;
+    __shared__ int ts_sh[kMaxExperts + 2];
+    __shared__ int rb_sh[kMaxExperts + 1];
+    __shared__ int rc_sh[kMaxExperts + 1];
+    __shared__ float amax_sh[2][kBM];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (p.single_rows > 0) {
+        if (threadIdx.x == 0) {
+            ts_sh[0] = 0;
+            ts_sh[1] = ((p.single_rows + kBM - 1) / kBM) * p.n_tiles_s;
+            rb_sh[0] = 0;
+            rc_sh[0] = p.single_rows;
+        }
+    } else {
+        for (int i = threadIdx.x; i <= p.G; i += blockDim.x) {
+            ts_sh[i] = p.tile_start[i];
+            if (i < p.G) {
+                rb_sh[i] = p.row_base[i];
+                rc_sh[i] = p.row_count[i];
+            }
+        }
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull_bar[b], 1);
+            mbar_init(&tempty_bar[b], 8);
+        }
+        mbar_init(&drain_bar, 1);
+        abort_sh = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+    const int total = ts_sh[p.G];
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_a_r);
+            prefetch_tensormap(&tm_a_s);
+            prefetch_tensormap(&tm_b0_r);
+            prefetch_tensormap(&tm_b1_r);
+            prefetch_tensormap(&tm_b0_s);
+            prefetch_tensormap(&tm_b1_s);
+            int stage = 0;
+            uint32_t phase = 0, pend = 0, pend_par = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                Tile ti;
+                decode_tile(t, ts_sh, rb_sh, rc_sh, p, kMode, ti);
+                const CUtensorMap* ma = ti.shared ? &tm_a_s : &tm_a_r;
+                const CUtensorMap* mb0 = ti.shared ? &tm_b0_s : &tm_b0_r;
+                const CUtensorMap* mb1 = ti.shared ? &tm_b1_s : &tm_b1_r;
+                const int b1_row = (kMode == kModeUp) ? ti.b_row0 : ti.b_row0 + 128;
+                for (int kb = 0; kb < ti.kb; ++kb) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, p.status, 0x10)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + stage * kStageBytes;
+                    uint8_t* sb = sa + kStageBytesA;
+                    mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
+                    const int kx = kb * (kFp8 ? 128 : 64);
+                    tma_load_2d(sa, ma, &full_bar[stage], kx, ti.a_row0);
+                    tma_load_2d(sb, mb0, &full_bar[stage], kx, ti.b_row0);
+                    tma_load_2d(sb + 128 * 128, mb1, &full_bar[stage], kx, b1_row);
+                    pend |= 1u << stage;
+                    pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok)
+                for (int s = 0; s < kStages; ++s)
+                    if ((pend >> s) & 1u) drain_wait(&full_bar[s], (pend_par >> s) & 1u);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = instr_desc(kFp8, kBM, kBN);
+            int stage = 0, abuf = 0;
+            uint32_t phase = 0, aphase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+                Tile ti;
+                decode_tile(t, ts_sh, rb_sh, rc_sh, p, kMode, ti);
+                for (int kb = 0; kb < ti.kb; ++kb) {
+                    if (kFp8 || kb == 0) {
+                        if (!mbar_wait(&tempty_bar[abuf], aphase ^ 1u, &abort_sh, p.status, 0x20)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    if (!mbar_wait(&full_bar[stage], phase, &abort_sh, p.status, 0x21)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+                    const uint64_t ad = smem_desc_sw128(sa);
+                    const uint64_t bd = smem_desc_sw128(sa + kStageBytesA);
+                    const uint32_t dt = tmem + static_cast<uint32_t>(abuf * kBN);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma<kFp8>(dt, ad + 2 * ks, bd + 2 * ks, idesc, kFp8 ? (ks > 0) : (kb > 0 || ks > 0));
+                    umma_commit(&empty_bar[stage]);
+                    if (kFp8 || kb == ti.kb - 1) {
+                        umma_commit(&tfull_bar[abuf]);
+                        abuf ^= 1;
+                        if (abuf == 0) aphase ^= 1u;
+                    }
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            umma_commit(&drain_bar);
+            drain_wait(&drain_bar, 0);
+        }
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int c = (warp - 2) >> 2;
+        const int r = q * 32 + lane;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(q * 32) << 16);
+        int abuf = 0;
+        uint32_t aphase = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+            Tile ti;
+            decode_tile(t, ts_sh, rb_sh, rc_sh, p, kMode, ti);
+            const int grow = ti.a_row0 + r;
+            const bool valid = r < ti.rows_valid;
+            uint8_t* out = static_cast<uint8_t*>(ti.shared ? p.out_s : p.out_r);
+            const size_t out_ld = static_cast<size_t>(ti.shared ? p.out_ld_s : p.out_ld_r);
+            if constexpr (kFp8) {
+                float acc[128];
+#pragma unroll
+                for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+                const float* as = ti.shared ? p.as_s : p.as_r;
+                const size_t as_ld = static_cast<size_t>(ti.shared ? p.as_ld_s : p.as_ld_r);
+                const int bcols = ti.shared ? p.bs_cols_s : p.bs_cols_r;
+                const int brow = (ti.shared ? 0 : ti.g * p.bs_rows_r) + (kMode == kModeUp ? ti.nt : 2 * ti.nt + c);
+                const float* sc0 = (ti.shared ? p.bs0_s : p.bs0_r) + static_cast<size_t>(brow) * bcols;
+                const float* sc1 = (ti.shared ? p.bs1_s : p.bs1_r) + static_cast<size_t>(brow) * bcols;
+                bool ok = true;
+                for (int kb = 0; kb < ti.kb; ++kb) {
+                    if (!mbar_wait(&tfull_bar[abuf], aphase, &abort_sh, p.status, 0x30)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float sa = as[static_cast<size_t>(kb) * as_ld + grow];
+                    const float f0 = sa * __ldg(sc0 + kb);
+                    const float f1 = (kMode == kModeUp) ? sa * __ldg(sc1 + kb) : f0;
+                    const uint32_t base = tl + static_cast<uint32_t>(abuf * kBN);
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        const int col = (kMode == kModeUp) ? ((ch < 2 ? 0 : 128) + 64 * c + 32 * (ch & 1))
+                                                           : (128 * c + 32 * ch);
+                        uint32_t v[32];
+                        tmem_ld32(base + col, v);
+                        tmem_wait_ld();
+                        const float f = (ch < 2) ? f0 : f1;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) acc[ch * 32 + j] = fmaf(__uint_as_float(v[j]), f, acc[ch * 32 + j]);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty_bar[abuf]);
+                    abuf ^= 1;
+                    if (abuf == 0) aphase ^= 1u;
+                }
+                if (!ok) break;
+                if constexpr (kMode == kModeUp) {
+                    // h = bf16(silu(g) * u) for I-columns nt*128 + 64c + j, then the 1x128 FP8 quant of h
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) {
+                        acc[j] = silu_mul(acc[j], acc[64 + j]);
+                        amax = fmaxf(amax, fabsf(acc[j]));
+                    }
+                    amax_sh[c][r] = amax;
+                    named_bar_sync(1, 256);
+                    amax = fmaxf(amax, amax_sh[c ^ 1][r]);
+                    named_bar_sync(1, 256);
+                    const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+                    if (valid) {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            uint32_t word = 0;
+                            if (amax > 0.0f) {
+#pragma unroll
+                                for (int b = 0; b < 4; ++b) {
+                                    const uint32_t code =
+                                        __nv_cvt_float_to_fp8(__fdiv_rn(acc[4 * i + b], sc), __NV_SATFINITE, __NV_E4M3);
+                                    word |= code << (8 * b);
+                                }
+                            }
+                            w[i] = word;
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(grow) * out_ld + ti.nt * 128 + 64 * c);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                        if (c == 0) {
+                            float* os = ti.shared ? p.outs_s : p.outs_r;
+                            const size_t os_ld = static_cast<size_t>(ti.shared ? p.outs_ld_s : p.outs_ld_r);
+                            os[static_cast<size_t>(ti.nt) * os_ld + grow] = sc;
+                        }
+                    }
+                } else {
+                    if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(grow) * out_ld + ti.nt * 256 + 128 * c) * 2);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            dst[i] = make_uint4(pack2(acc[8 * i], acc[8 * i + 1]), pack2(acc[8 * i + 2], acc[8 * i + 3]),
+                                                pack2(acc[8 * i + 4], acc[8 * i + 5]), pack2(acc[8 * i + 6], acc[8 * i + 7]));
+                    }
+                }
+            } else {
+                // bf16: the whole K accumulated in TMEM buffer abuf
+                if (!mbar_wait(&tfull_bar[abuf], aphase, &abort_sh, p.status, 0x31)) break;
+                tc_fence_after();
+                const uint32_t base = tl + static_cast<uint32_t>(abuf * kBN);
+                if constexpr (kMode == kModeUp) {
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t vg[32], vu[32];
+                        tmem_ld32(base + 64 * c + 32 * hh, vg);
+                        tmem_ld32(base + 128 + 64 * c + 32 * hh, vu);
+                        tmem_wait_ld();
+                        if (valid) {
+                            uint4* dst = reinterpret_cast<uint4*>(
+                                out + (static_cast<size_t>(grow) * out_ld + ti.nt * 128 + 64 * c + 32 * hh) * 2);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                float h[8];
+#pragma unroll
+                                for (int b = 0; b < 8; ++b)
+                                    h[b] = silu_mul(__uint_as_float(vg[8 * i + b]), __uint_as_float(vu[8 * i + b]));
+                                dst[i] = make_uint4(pack2(h[0], h[1]), pack2(h[2], h[3]), pack2(h[4], h[5]), pack2(h[6], h[7]));
+                            }
+                        }
+                    }
+                } else if constexpr (kMode == kModeDown) {
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t v[32];
+                        tmem_ld32(base + 128 * c + 32 * ch, v);
+                        tmem_wait_ld();
+                        if (valid) {
+                            uint4* dst = reinterpret_cast<uint4*>(
+                                out + (static_cast<size_t>(grow) * out_ld + ti.nt * 256 + 128 * c + 32 * ch) * 2);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                dst[i] = make_uint4(pack2(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
+                                                    pack2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                                                    pack2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                                                    pack2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+                        }
+                    }
+                } else {
+                    // router logits, float32, columns < n_valid_cols (a multiple of 8)
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t v[32];
+                        tmem_ld32(base + 128 * c + 32 * ch, v);
+                        tmem_wait_ld();
+                        const int col0 = 128 * c + 32 * ch;
+                        if (valid) {
+                            float* dst = reinterpret_cast<float*>(out + (static_cast<size_t>(grow) * out_ld + col0) * 4);
+                            if ((p.n_valid_cols & 3) == 0) {        // rows 16-byte aligned: vector stores
+#pragma unroll
+                                for (int i = 0; i < 8; ++i)
+                                    if (col0 + 4 * i < p.n_valid_cols)
+                                        reinterpret_cast<float4*>(dst)[i] =
+                                            make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                        __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 32; ++i)
+                                    if (col0 + i < p.n_valid_cols) dst[i] = __uint_as_float(v[i]);
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty_bar[abuf]);
+                abuf ^= 1;
+                if (abuf == 0) aphase ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <bool kFp8, int kMode>
+cudaError_t launch_one(const TensorMaps& m, const GemmParams& p, int grid, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kFp8, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+    if (e != cudaSuccess) return e;
+    gemm_kernel<kFp8, kMode><<<grid, kGemmThreads, kSmemBytes, s>>>(m.a_r, m.a_s, m.b0_r, m.b1_r, m.b0_s, m.b1_s, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(int mode, bool fp8, const TensorMaps& maps, const GemmParams& p, int grid, cudaStream_t s) {
+    if (fp8) {
+        if (mode == kModeUp) return launch_one<true, kModeUp>(maps, p, grid, s);
+        if (mode == kModeDown) return launch_one<true, kModeDown>(maps, p, grid, s);
+        return cudaErrorInvalidValue;
+    }
+    if (mode == kModeUp) return launch_one<false, kModeUp>(maps, p, grid, s);
+    if (mode == kModeDown) return launch_one<false, kModeDown>(maps, p, grid, s);
+    return launch_one<false, kModeLogits>(maps, p, grid, s);
+}
+
+}  // namespace moe

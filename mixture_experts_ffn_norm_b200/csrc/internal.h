@@ -1,0 +1,83 @@
+// Internal declarations shared by the .cu files of libmoe: workspace layout, grouped-GEMM
+// parameters and the host-side launchers of each kernel.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kBM = 128;          // rows of A per GEMM tile (tokens)
+constexpr int kBN = 256;          // columns (weight rows) per GEMM tile
+constexpr int kStageBytesA = kBM * 128;
+constexpr int kStageBytesB = kBN * 128;
+constexpr int kStages = 4;
+constexpr int kGemmThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kMaxExperts = 256;
+constexpr int kRouteChunk = 2048;  // (token, slot) entries per block in the routing kernels
+
+enum GemmMode : int { kModeLogits = 0, kModeUp = 1, kModeDown = 2 };
+
+// Byte offsets of every region of the caller's workspace.
+struct Layout {
+    int T, d, I, E, k, Is, Tpad, R, KBd, KBi, KBs, nchunks;
+    bool fp8, act8;
+    size_t status, xn, xq, xs, logits, idx, w, flag, flag_list, counts, offsets, row_base, row_count,
+        ts_up, ts_down, chunk_hist, row_of, row_token, a_perm, as_perm, h, hs, h_sh, hs_sh, y, y_sh, total;
+};
+
+bool make_layout(const moe_config_t& c, Layout& L);
+
+// Parameters of the persistent grouped GEMM.  Groups 0..G-2 (or 0..G-1 without a shared expert)
+// are routed experts whose rows sit at row_base[g] in the permuted A; the last group is the shared
+// expert over all T tokens in token order.  Everything group-dependent is read on the device, so
+// the host never learns the routing.
+struct GemmParams {
+    int G;                      // number of groups
+    int has_shared;             // last group is the shared expert
+    int single_rows;            // > 0: one shared-style group of this many rows, no device arrays
+    const int* tile_start;      // [G + 1] cumulative tile counts
+    const int* row_base;        // [G]
+    const int* row_count;       // [G]
+    int n_tiles_r, n_tiles_s;   // N tiles of a routed / the shared group
+    int kb_r, kb_s;             // K stages of a routed / the shared group
+    int b_rows_per_expert;      // rows of one routed expert in the B tensor
+    // activation scales, transposed [K/128][ld] (FP8 only)
+    const float* as_r; const float* as_s;
+    int as_ld_r, as_ld_s;
+    // weight block scales (FP8 only): routed [E][rows/128][cols/128], shared [rows/128][cols/128]
+    const float* bs0_r; const float* bs1_r; const float* bs0_s; const float* bs1_s;
+    int bs_cols_r, bs_cols_s, bs_rows_r;
+    // outputs: row-major with row strides (elements) out_ld_*; output scales transposed [N/128][ld]
+    void* out_r; void* out_s;
+    int out_ld_r, out_ld_s;
+    float* outs_r; float* outs_s;
+    int outs_ld_r, outs_ld_s;
+    int n_valid_cols;           // logits: columns actually stored (E)
+    uint32_t* status;
+};
+
+struct TensorMaps {
+    CUtensorMap a_r, a_s, b0_r, b1_r, b0_s, b1_s;
+};
+
+// tensor-map encoding (driver entry point fetched at run time; no libcuda link)
+bool encode_map_2d(CUtensorMap* map, const void* base, bool fp8, uint64_t inner, uint64_t rows);
+
+cudaError_t launch_norm(const Layout& L, const void* x, const void* residual, const float* g, float eps,
+                        void* residual_out, uint8_t* ws, cudaStream_t s);
+cudaError_t launch_gemm(int mode, bool fp8, const TensorMaps& maps, const GemmParams& p, int grid,
+                        cudaStream_t s);
+cudaError_t launch_topk(const Layout& L, const float* gate_bias, float tau, uint8_t* ws, cudaStream_t s);
+cudaError_t launch_recheck(const Layout& L, const void* gate_w, const float* gate_bias, uint8_t* ws,
+                           cudaStream_t s);
+cudaError_t launch_route(const Layout& L, int ntu_r, int ntu_s, int ntd_r, int ntd_s, uint8_t* ws,
+                         cudaStream_t s);
+cudaError_t launch_combine(const Layout& L, void* out, uint8_t* ws, cudaStream_t s);
+
+int num_sms();
+
+}  // namespace moe

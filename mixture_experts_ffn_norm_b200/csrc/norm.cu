@@ -1,0 +1,165 @@
+// ffn_norm: RMSNorm with the residual add fused in, plus the per-token 1x128 FP8 quant of the
+// normed activations that the FP8 expert GEMMs consume.
+//
+// "MoE update" page, RMSNorm.forward excerpt: s = x.float() + residual.float();
+// var = mean(s^2); s * rsqrt(var + eps); weight * s; the normed value and the new residual are
+// cast back to x's dtype.  The mean is taken as the exact sum of the squares rounded to double
+// (double-double accumulation: every float32 square is exact in double, the TwoSum error terms
+// carry the rest), divided by d in double and rounded to float32, so the result does not depend
+// on the reduction order.  rsqrt = IEEE sqrt then IEEE divide, and no multiply is contracted
+// into an FMA, so every float32 step is the correctly rounded one.
+//
+// One CTA per token, 128 threads, 16-byte vector loads and stores; the token's float32 sums stay
+// in shared memory between the two passes.  Memory-bound: reads 4d bytes, writes 4d (+d + d/32).
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(a));
+    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(b));
+    return lo | (hi << 16);
+}
+
+// error-free sum of two doubles: (s, e) with s + e == a + b exactly
+__device__ __forceinline__ void two_sum(double a, double b, double& s, double& e) {
+    s = __dadd_rn(a, b);
+    const double bb = __dsub_rn(s, a);
+    e = __dadd_rn(__dsub_rn(a, __dsub_rn(s, bb)), __dsub_rn(b, bb));
+}
+
+__device__ __forceinline__ void dd_add(double& hi, double& lo, double hi2, double lo2) {
+    double s, e;
+    two_sum(hi, hi2, s, e);
+    hi = s;
+    lo = __dadd_rn(lo, __dadd_rn(lo2, e));
+}
+
+constexpr int kNormThreads = 128;
+
+__global__ void __launch_bounds__(kNormThreads)
+norm_kernel(const uint4* __restrict__ x, const uint4* __restrict__ res, const float* __restrict__ gain,
+            float eps, int d, int Tpad, uint4* __restrict__ res_out, uint4* __restrict__ xn,
+            uint2* __restrict__ xq, float* __restrict__ xs) {
+    extern __shared__ float s_sh[];                 // d floats: s = x + residual
+    __shared__ double red_hi[kNormThreads / 32], red_lo[kNormThreads / 32];
+    __shared__ float rinv_sh;
+    const int t = blockIdx.x;
+    const int nv = d >> 3;
+    const size_t row = static_cast<size_t>(t) * nv;
+
+    double hi = 0.0, lo = 0.0;
+    for (int v = threadIdx.x; v < nv; v += kNormThreads) {
+        const uint4 xa = x[row + v];
+        const uint32_t xw[4] = {xa.x, xa.y, xa.z, xa.w};
+        float s[8];
+        if (res) {
+            const uint4 ra = res[row + v];
+            const uint32_t rw[4] = {ra.x, ra.y, ra.z, ra.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                s[2 * i] = __fadd_rn(bf16_lo(xw[i]), bf16_lo(rw[i]));
+                s[2 * i + 1] = __fadd_rn(bf16_hi(xw[i]), bf16_hi(rw[i]));
+            }
+            res_out[row + v] = make_uint4(pack_bf16(s[0], s[1]), pack_bf16(s[2], s[3]), pack_bf16(s[4], s[5]),
+                                          pack_bf16(s[6], s[7]));
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                s[2 * i] = bf16_lo(xw[i]);
+                s[2 * i + 1] = bf16_hi(xw[i]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            s_sh[v * 8 + i] = s[i];
+            const double p = __dmul_rn(static_cast<double>(s[i]), static_cast<double>(s[i]));  // exact
+            double sum, err;
+            two_sum(hi, p, sum, err);
+            hi = sum;
+            lo = __dadd_rn(lo, err);
+        }
+    }
+    // block reduction of the double-double partial sums
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const double h2 = __shfl_xor_sync(0xFFFFFFFFu, hi, off);
+        const double l2 = __shfl_xor_sync(0xFFFFFFFFu, lo, off);
+        dd_add(hi, lo, h2, l2);
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        red_hi[warp] = hi;
+        red_lo[warp] = lo;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double H = red_hi[0], Lo = red_lo[0];
+        for (int w = 1; w < kNormThreads / 32; ++w) dd_add(H, Lo, red_hi[w], red_lo[w]);
+        const double ss = __dadd_rn(H, Lo);                                  // RN64 of the sum
+        const float var = __double2float_rn(__ddiv_rn(ss, static_cast<double>(d)));
+        const float v = __fadd_rn(var, eps);
+        rinv_sh = __fdiv_rn(1.0f, __fsqrt_rn(v));
+    }
+    __syncthreads();
+    const float rinv = rinv_sh;
+
+    for (int v = threadIdx.x; v < nv; v += kNormThreads) {
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float tt = __fmul_rn(s_sh[v * 8 + i], rinv);               // x * rsqrt(var + eps)
+            y[i] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(gain[v * 8 + i], tt)));  // (weight * x) -> bf16
+        }
+        xn[row + v] = make_uint4(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]), pack_bf16(y[4], y[5]),
+                                 pack_bf16(y[6], y[7]));
+        if (xq) {
+            // 1x128 group = 16 consecutive vectors = 16 consecutive lanes of this warp
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(y[i]));
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+            const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+            uint32_t q[2] = {0u, 0u};
+            if (amax > 0.0f) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t c = __nv_cvt_float_to_fp8(__fdiv_rn(y[i], sc), __NV_SATFINITE, __NV_E4M3);
+                    q[i >> 2] |= c << (8 * (i & 3));
+                }
+            }
+            xq[row + v] = make_uint2(q[0], q[1]);
+            if ((v & 15) == 0) xs[static_cast<size_t>(v >> 4) * Tpad + t] = sc;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_norm(const Layout& L, const void* x, const void* residual, const float* g, float eps,
+                        void* residual_out, uint8_t* ws, cudaStream_t s) {
+    const size_t smem = static_cast<size_t>(L.d) * sizeof(float);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(norm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+    }
+    norm_kernel<<<L.T, kNormThreads, smem, s>>>(
+        static_cast<const uint4*>(x), static_cast<const uint4*>(residual), g, eps, L.d, L.Tpad,
+        static_cast<uint4*>(residual_out), reinterpret_cast<uint4*>(ws + L.xn),
+        L.act8 ? reinterpret_cast<uint2*>(ws + L.xq) : nullptr,
+        L.act8 ? reinterpret_cast<float*>(ws + L.xs) : nullptr);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,181 @@
+// Token permutation by expert, with no host synchronisation.
+//
+// The pages' loop ("MoE update" page, MoE.forward excerpt) counts tokens per expert with
+// torch.bincount(...).tolist() -- a device-to-host copy -- and gathers each expert's
+// (token, slot) pairs with torch.where.  Here the same grouping is built on the device:
+//   hist    : per chunk of 2048 (token, slot) entries, a shared-memory histogram over experts;
+//   scan    : per expert, exclusive prefix over chunks (stable order) and over experts of the
+//             counts padded to the 128-row GEMM tile; the grouped GEMMs' tile tables;
+//   scatter : every entry gets its row in the permuted order (token order inside an expert,
+//             so the permutation is deterministic);
+//   gather  : the permuted activation rows (FP8 codes or bf16) and their group scales are
+//             copied next to each other so a TMA box of 128 rows is one expert's tile.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRouteThreads = 256;
+
+__global__ void __launch_bounds__(kRouteThreads)
+hist_kernel(const int* __restrict__ idx, int N, int E, int* __restrict__ chunk_hist, uint32_t* status) {
+    __shared__ int h[kMaxExperts];
+    for (int e = threadIdx.x; e < kMaxExperts; e += kRouteThreads) h[e] = 0;
+    __syncthreads();
+    const int c = blockIdx.x;
+    const int end = min(N, (c + 1) * kRouteChunk);
+    for (int i = c * kRouteChunk + threadIdx.x; i < end; i += kRouteThreads) {
+        const int e = idx[i];
+        if (e >= 0 && e < E) atomicAdd(&h[e], 1);
+        else latch_error(status, kErrCheck, 0x100);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kRouteThreads) chunk_hist[static_cast<size_t>(c) * E + e] = h[e];
+}
+
+// block-wide exclusive scan of one int per thread (256 threads); returns the total in *total
+__device__ int block_exclusive_scan(int v, int* sh, int* total) {
+    const int tid = threadIdx.x;
+    sh[tid] = v;
+    __syncthreads();
+    for (int off = 1; off < kRouteThreads; off <<= 1) {
+        const int add = tid >= off ? sh[tid - off] : 0;
+        __syncthreads();
+        sh[tid] += add;
+        __syncthreads();
+    }
+    const int incl = sh[tid];
+    *total = sh[kRouteThreads - 1];
+    __syncthreads();
+    return incl - v;
+}
+
+__global__ void __launch_bounds__(kRouteThreads)
+scan_kernel(int* __restrict__ chunk_hist, int nchunks, int E, int T, int has_shared, int ntu_r, int ntu_s,
+            int ntd_r, int ntd_s, int* __restrict__ counts, int* __restrict__ offsets, int* __restrict__ row_base,
+            int* __restrict__ row_count, int* __restrict__ ts_up, int* __restrict__ ts_down) {
+    __shared__ int sh[kRouteThreads];
+    const int e = threadIdx.x;
+    int cnt = 0;
+    if (e < E) {
+        for (int c = 0; c < nchunks; ++c) {
+            const int v = chunk_hist[static_cast<size_t>(c) * E + e];
+            chunk_hist[static_cast<size_t>(c) * E + e] = cnt;   // exclusive base of chunk c
+            cnt += v;
+        }
+    }
+    const int mtiles = (cnt + kBM - 1) / kBM;
+    int tot_rows, tot_up, tot_down;
+    const int off = block_exclusive_scan(mtiles * kBM, sh, &tot_rows);
+    const int tu = block_exclusive_scan(mtiles * ntu_r, sh, &tot_up);
+    const int td = block_exclusive_scan(mtiles * ntd_r, sh, &tot_down);
+    if (e < E) {
+        counts[e] = cnt;
+        offsets[e] = off;
+        row_base[e] = off;
+        row_count[e] = cnt;
+        ts_up[e] = tu;
+        ts_down[e] = td;
+    }
+    if (e == 0) {
+        offsets[E] = tot_rows;
+        ts_up[E] = tot_up;
+        ts_down[E] = tot_down;
+        if (has_shared) {
+            const int mt = (T + kBM - 1) / kBM;
+            row_base[E] = 0;
+            row_count[E] = T;
+            ts_up[E + 1] = tot_up + mt * ntu_s;
+            ts_down[E + 1] = tot_down + mt * ntd_s;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kRouteThreads)
+scatter_kernel(const int* __restrict__ idx, int N, int E, int k, const int* __restrict__ chunk_base,
+               const int* __restrict__ offsets, int* __restrict__ row_of, int* __restrict__ row_token) {
+    __shared__ int run_base[kMaxExperts];
+    __shared__ int wcnt[kRouteThreads / 32][kMaxExperts];
+    const int c = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < kMaxExperts; e += kRouteThreads) {
+        run_base[e] = e < E ? offsets[e] + chunk_base[static_cast<size_t>(c) * E + e] : 0;
+#pragma unroll
+        for (int w = 0; w < kRouteThreads / 32; ++w) wcnt[w][e] = 0;
+    }
+    __syncthreads();
+    const int end = min(N, (c + 1) * kRouteChunk);
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int base = c * kRouteChunk; base < end; base += kRouteThreads) {
+        const int i = base + threadIdx.x;
+        const bool valid = i < end;
+        int e = valid ? idx[i] : -1;
+        if (e < 0 || e >= E) e = -1;
+        const uint32_t m = __match_any_sync(0xFFFFFFFFu, e);
+        const int lane_rank = __popc(m & lt_mask);
+        const bool leader = (__ffs(m) - 1) == lane;
+        if (e >= 0 && leader) wcnt[warp][e] = __popc(m);
+        __syncthreads();
+        if (e >= 0) {
+            int rank = lane_rank;
+            for (int w = 0; w < warp; ++w) rank += wcnt[w][e];
+            const int pos = run_base[e] + rank;
+            row_of[i] = pos;
+            row_token[pos] = i / k;
+        }
+        __syncthreads();
+        if (e >= 0 && leader) {
+            atomicAdd(&run_base[e], __popc(m));
+            wcnt[warp][e] = 0;
+        }
+        __syncthreads();
+    }
+}
+
+// One warp per permuted row: copy the token's activation row and its group scales.
+__global__ void __launch_bounds__(kRouteThreads)
+gather_kernel(const int* __restrict__ row_token, const int* __restrict__ offsets, int E,
+              const uint4* __restrict__ src, int row_vecs, uint4* __restrict__ dst, const float* __restrict__ xs,
+              int Tpad, float* __restrict__ as, int R, int KB) {
+    const int total = offsets[E];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int p = blockIdx.x * (kRouteThreads / 32) + warp; p < total; p += gridDim.x * (kRouteThreads / 32)) {
+        const int t = row_token[p];
+        if (t < 0) continue;
+        const uint4* s = src + static_cast<size_t>(t) * row_vecs;
+        uint4* d = dst + static_cast<size_t>(p) * row_vecs;
+        for (int v = lane; v < row_vecs; v += 32) d[v] = s[v];
+        if (as)
+            for (int kb = lane; kb < KB; kb += 32) as[static_cast<size_t>(kb) * R + p] = xs[static_cast<size_t>(kb) * Tpad + t];
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_route(const Layout& L, int ntu_r, int ntu_s, int ntd_r, int ntd_s, uint8_t* ws, cudaStream_t s) {
+    const int N = L.T * L.k;
+    int* idx = reinterpret_cast<int*>(ws + L.idx);
+    int* chunk = reinterpret_cast<int*>(ws + L.chunk_hist);
+    uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+    hist_kernel<<<L.nchunks, kRouteThreads, 0, s>>>(idx, N, L.E, chunk, status);
+    scan_kernel<<<1, kRouteThreads, 0, s>>>(chunk, L.nchunks, L.E, L.T, L.Is > 0, ntu_r, ntu_s, ntd_r, ntd_s,
+                                            reinterpret_cast<int*>(ws + L.counts), reinterpret_cast<int*>(ws + L.offsets),
+                                            reinterpret_cast<int*>(ws + L.row_base),
+                                            reinterpret_cast<int*>(ws + L.row_count), reinterpret_cast<int*>(ws + L.ts_up),
+                                            reinterpret_cast<int*>(ws + L.ts_down));
+    scatter_kernel<<<L.nchunks, kRouteThreads, 0, s>>>(idx, N, L.E, L.k, chunk, reinterpret_cast<int*>(ws + L.offsets),
+                                                       reinterpret_cast<int*>(ws + L.row_of),
+                                                       reinterpret_cast<int*>(ws + L.row_token));
+    const int row_bytes = L.act8 ? L.d : 2 * L.d;
+    const int grid = 4 * num_sms();
+    gather_kernel<<<grid, kRouteThreads, 0, s>>>(
+        reinterpret_cast<const int*>(ws + L.row_token), reinterpret_cast<const int*>(ws + L.offsets), L.E,
+        reinterpret_cast<const uint4*>(ws + (L.act8 ? L.xq : L.xn)), row_bytes / 16,
+        reinterpret_cast<uint4*>(ws + L.a_perm), L.act8 ? reinterpret_cast<const float*>(ws + L.xs) : nullptr,
+        L.Tpad, L.act8 ? reinterpret_cast<float*>(ws + L.as_perm) : nullptr, L.R, L.KBd);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,157 @@
+"""Helpers shared by the GPU parity tests: run the CUDA path through the C ABI, run the oracle on
+host copies of the same seeded inputs, and compare with the stated criteria.
+
+Criteria (per workload):
+  residual_out          bit-exact
+  xn (normed, bf16)     bit-exact;  xq / xs (FP8 activation quant) bit-exact
+  routing sets          bit-exact for tokens whose oracle margin (k-th minus (k+1)-th score) is
+                        >= 1e-6; the others are counted and reported
+  counts                equal to the bincount of the GPU's own indices
+  routing weights       <= 1e-5 relative
+  out                   max |err| <= 2e-2 * RMS(oracle out) over the checked elements
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import torch
+
+import mixture_experts_ffn_norm_b200 as moe
+import oracle
+import synthetic
+from oracle import bf16_bits_to_f64
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+MARGIN_EXEMPT = 1e-6
+OUT_TOL = 2e-2
+W_RTOL = 1e-5
+
+
+def c5_alpha() -> float:
+    with open(os.path.join(GOLDEN, "c5_alpha.json")) as f:
+        return json.load(f)["alpha"]
+
+
+def inputs_for(shape, device="cuda", **kw):
+    alpha = c5_alpha() if shape.zipf_bias else None
+    return synthetic.generate(shape, device=device, alpha=alpha, **kw)
+
+
+def bits_np(t: torch.Tensor) -> np.ndarray:
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+class GpuRun:
+    """One moe_forward through the C ABI plus every debug export, copied to the host."""
+
+    def __init__(self, shape, inp: dict, residual=True, in_place=False, tie_tau=0.0, cfg=None):
+        self.shape = shape
+        self.cfg = cfg or moe.Config.from_shape(shape, tie_tau=tie_tau)
+        dev = inp["x"].device
+        T, d, k, E = self.cfg.num_tokens, self.cfg.dim, self.cfg.top_k, self.cfg.n_experts
+        self.layer = moe.MoELayer(self.cfg, {n: v for n, v in inp.items() if n not in ("x", "residual")}, device=dev)
+        x = inp["x"]
+        r = inp["residual"].clone() if residual else None
+        out = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+        ro = (r if in_place else torch.empty_like(x)) if residual else None
+        self.layer.forward(x, r, out, ro)
+        st = moe.moe_get_status(self.layer.workspace)
+        assert st == moe.MOE_OK, moe.status_string(st)
+        idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+        w = torch.empty(T, k, dtype=torch.float32, device=dev)
+        cnt = torch.empty(E, dtype=torch.int32, device=dev)
+        tie = torch.empty(T, dtype=torch.uint8, device=dev)
+        moe.moe_debug_routing(self.cfg, self.layer.workspace, idx, w, cnt, tie)
+        xn = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+        fp8 = self.cfg.wtype == moe.MOE_W_FP8_E4M3_B128
+        xq = torch.empty(T, d, dtype=torch.uint8, device=dev) if fp8 else None
+        xs = torch.empty(d // 128, T, dtype=torch.float32, device=dev) if fp8 else None
+        moe.moe_debug_norm(self.cfg, self.layer.workspace, xn, xq, xs)
+        torch.cuda.synchronize()
+        self.out = bits_np(out)
+        self.residual_out = bits_np(ro) if residual else None
+        self.idx, self.w, self.counts, self.near_tie = idx.cpu().numpy(), w.cpu().numpy(), cnt.cpu().numpy(), tie.cpu().numpy()
+        self.xn = bits_np(xn)
+        self.xq = None if xq is None else xq.cpu().numpy()
+        self.xs = None if xs is None else xs.cpu().numpy()
+
+
+def check_routing(run: GpuRun, ref: dict, tokens: np.ndarray, report: dict):
+    """Routing sets, weights and counts for the tokens the oracle evaluated."""
+    k = run.cfg.top_k
+    g_idx = run.idx[tokens]
+    o_idx = ref["idx"]
+    exempt = ref["margin"] < MARGIN_EXEMPT
+    same = np.all(np.sort(g_idx, 1) == np.sort(o_idx, 1), axis=1)
+    bad = np.nonzero(~same & ~exempt)[0]
+    report["routing_tokens"] = int(len(tokens))
+    report["near_tie_exempt"] = int(exempt.sum())
+    report["near_tie_exempt_differing"] = int((~same & exempt).sum())
+    report["gpu_rechecked"] = int(run.near_tie.sum())
+    assert len(bad) == 0, f"routing differs for tokens {tokens[bad][:10]} (margins {ref['margin'][bad][:5]})"
+    # weights, matched by expert id
+    ok = same & ~exempt
+    if ok.any():
+        og = np.argsort(g_idx[ok], 1)
+        oo = np.argsort(o_idx[ok], 1)
+        gw = np.take_along_axis(run.w[tokens][ok].astype(np.float64), og, 1)
+        ow = np.take_along_axis(ref["w"][ok], oo, 1)
+        rel = np.abs(gw - ow) / np.abs(ow)
+        report["weights_max_rel"] = float(rel.max())
+        assert rel.max() <= W_RTOL, rel.max()
+    # indices distinct per token, counts == bincount of the GPU's own indices
+    assert np.all(np.sort(run.idx, 1)[:, 1:] != np.sort(run.idx, 1)[:, :-1]) if k > 1 else True
+    assert np.array_equal(run.counts, np.bincount(run.idx.ravel(), minlength=run.cfg.n_experts))
+    assert run.counts.sum() == run.cfg.num_tokens * k
+
+
+def check_norm(run: GpuRun, ref: dict, tokens: np.ndarray, report: dict):
+    if run.residual_out is not None:
+        assert np.array_equal(run.residual_out[tokens], ref["residual_out"]), "residual_out not bit-exact"
+    assert np.array_equal(run.xn[tokens], ref["xn"]), "xn not bit-exact"
+    rel = np.abs(bf16_bits_to_f64(run.xn[tokens]) - ref["xn64"]) / np.maximum(np.abs(ref["xn64"]), 1e-30)
+    report["xn_vs_f64_max_rel"] = float(rel.max())
+    if run.xq is not None:
+        for p, t in enumerate(tokens[:64]):
+            q, sc, _ = oracle.act_quant(bf16_bits_to_f64(ref["xn"][p]))
+            assert np.array_equal(run.xq[t], q), f"xq differs for token {t}"
+            assert np.array_equal(run.xs[:, t], sc), f"xs differs for token {t}"
+
+
+def check_out(run: GpuRun, ref: dict, tokens: np.ndarray, report: dict):
+    g = bf16_bits_to_f64(run.out[tokens])
+    o = bf16_bits_to_f64(ref["out"])
+    rms = float(np.sqrt(np.mean(o ** 2)))
+    err = float(np.abs(g - o).max())
+    report["out_rms"] = rms
+    report["out_max_err"] = err
+    report["out_max_err_over_rms"] = err / rms
+    report["out_bitexact_frac"] = float(np.mean(run.out[tokens] == ref["out"]))
+    assert np.all(np.isfinite(g))
+    assert err <= OUT_TOL * rms, f"max|err| {err} > {OUT_TOL} * RMS {rms}"
+
+
+def sample_tokens(run: GpuRun, ref_route: dict, n_random: int, seed: int = 0) -> np.ndarray:
+    """A seeded token sample that covers every expert the GPU routed to (greedy), every token with a
+    small margin, plus n_random others and the last token (ragged tail)."""
+    T, E = run.cfg.num_tokens, run.cfg.n_experts
+    rng = np.random.default_rng(seed)
+    chosen = set(np.nonzero(ref_route["margin"] < 1e-4)[0][:64].tolist())
+    chosen.add(T - 1)
+    covered = np.zeros(E, bool)
+    for t in chosen:
+        covered[run.idx[t]] = True
+    order = rng.permutation(T)
+    for t in order:
+        if covered.all():
+            break
+        if not covered[run.idx[t]].all():
+            chosen.add(int(t))
+            covered[run.idx[t]] = True
+    chosen.update(rng.choice(T, size=min(n_random, T), replace=False).tolist())
+    return np.array(sorted(chosen), dtype=np.int32)

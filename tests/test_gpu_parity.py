@@ -1,0 +1,151 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on the same seeded inputs.
+
+Small and ragged layers are compared on every token; the full-size workloads (decode, prefill,
+skewed routing) are run exactly as bench.py launches them and compared on a seeded token sample
+that covers every expert the GPU used, with routing checked on all tokens.
+"""
+import dataclasses
+import json
+
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_ffn_norm_b200 as moe
+import oracle
+import synthetic
+from harness import GpuRun, check_norm, check_out, check_routing, inputs_for, sample_tokens
+
+pytestmark = pytest.mark.gpu
+
+
+def _shape(**kw):
+    base = dict(name="t", T=300, d=512, I=256, E=16, k=4, n_shared=1, shared_inter=256, wtype="fp8", seed=21)
+    base.update(kw)
+    return synthetic.MoEShape(**base)
+
+
+def _full_check(shape, inp, report, residual=True, **kw):
+    run = GpuRun(shape, inp, residual=residual, **kw)
+    o = oracle.Oracle(shape, dict(inp, residual=inp["residual"] if residual else None))
+    ref = o.forward()
+    toks = np.arange(shape.T, dtype=np.int32)
+    check_norm(run, ref, toks, report)
+    check_routing(run, ref, toks, report)
+    check_out(run, ref, toks, report)
+    print(shape.name, json.dumps(report))
+    return run, ref
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.init()
+
+
+def test_tiny_layer_every_token():
+    shape = synthetic.CONFIGS["C1"]
+    _full_check(shape, inputs_for(shape), {})
+
+
+@pytest.mark.parametrize("wtype,T", [("fp8", 300), ("bf16", 200), ("fp8", 1), ("bf16", 129)])
+def test_ragged_layers_every_token(wtype, T):
+    shape = _shape(wtype=wtype, T=T, I=384 if wtype == "bf16" else 256)
+    _full_check(shape, inputs_for(shape), {})
+
+
+def test_no_residual_and_no_shared_expert():
+    shape = _shape(T=160, shared_inter=0, n_shared=0)
+    _full_check(shape, inputs_for(shape), {}, residual=False)
+
+
+def test_k_equals_E_and_zero_gate_ties():
+    shape = dataclasses.replace(synthetic.CONFIGS["C1"], k=8)
+    inp = inputs_for(shape)
+    _full_check(shape, inp, {})
+    inp["gate_w"] = torch.zeros_like(inp["gate_w"])
+    shape2 = dataclasses.replace(synthetic.CONFIGS["C1"], k=3)
+    run, ref = _full_check(shape2, inp, {})
+    assert np.all(run.idx == np.arange(3)) and np.allclose(run.w, 1 / 3)
+
+
+def test_skew_all_tokens_to_few_experts_and_empty_experts():
+    shape = _shape(T=520, k=2, E=16)
+    inp = inputs_for(shape)
+    b = torch.full((16,), -30.0, device="cuda")
+    b[5] = 30.0          # every token picks expert 5 ...
+    b[11] = 20.0         # ... and expert 11: two groups of 520 rows (5 M-tiles, ragged), 14 empty
+    inp["gate_bias"] = b
+    run, _ = _full_check(shape, inp, {})
+    assert run.counts[5] == 520 and run.counts[11] == 520 and run.counts.sum() == 1040
+
+
+def test_in_place_residual_and_determinism():
+    shape = _shape(T=256)
+    inp = inputs_for(shape)
+    a = GpuRun(shape, inp, in_place=True)
+    b = GpuRun(shape, inp)
+    assert np.array_equal(a.residual_out, b.residual_out)
+    assert np.array_equal(a.out, b.out) and np.array_equal(a.idx, b.idx)
+
+
+def test_token_permutation_and_identical_experts_on_gpu():
+    shape = _shape(T=256)
+    inp = inputs_for(shape)
+    perm = torch.randperm(shape.T, generator=torch.Generator().manual_seed(3)).cuda()
+    a = GpuRun(shape, inp)
+    inp_p = dict(inp, x=inp["x"][perm].contiguous(), residual=inp["residual"][perm].contiguous())
+    b = GpuRun(shape, inp_p)
+    p = perm.cpu().numpy()
+    assert np.array_equal(a.out[p], b.out)
+    assert np.array_equal(np.sort(a.idx[p], 1), np.sort(b.idx, 1))
+    # identical experts: the output no longer depends on which experts were chosen
+    inp_i = dict(inp)
+    for n in ("w1", "w3", "w2", "s1", "s3", "s2"):
+        inp_i[n] = inp[n][:1].expand_as(inp[n]).contiguous()
+    c = GpuRun(shape, inp_i)
+    d = GpuRun(shape, dict(inp_i, gate_w=(-inp["gate_w"].float()).to(torch.bfloat16)))
+    gc, gd = oracle.bf16_bits_to_f64(c.out), oracle.bf16_bits_to_f64(d.out)
+    assert np.abs(gc - gd).max() <= 2e-2 * np.sqrt(np.mean(gc ** 2))
+
+
+def test_workspace_and_argument_errors():
+    shape = _shape(T=64)
+    inp = inputs_for(shape)
+    cfg = moe.Config.from_shape(shape)
+    layer = moe.MoELayer(cfg, {n: v for n, v in inp.items() if n not in ("x", "residual")})
+    out = torch.empty(64, 512, dtype=torch.bfloat16, device="cuda")
+    ro = torch.empty_like(out)
+    small = layer.workspace[: layer.workspace.numel() - 1024]
+    rc = moe.moe_forward(cfg, inp["x"], inp["residual"], layer.t["norm_w"], layer.t["gate_w"], None, layer.wstruct,
+                         out, ro, small, check=False)
+    assert rc == moe.MOE_ERR_WORKSPACE
+    rc = moe.moe_forward(cfg, inp["x"], inp["residual"], layer.t["norm_w"], layer.t["gate_w"], None, layer.wstruct,
+                         inp["x"], ro, layer.workspace, check=False)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_get_status(layer.workspace) == moe.MOE_OK
+
+
+# ------------------------------------------------------------------------------------------------
+# the five workloads at full size, launched as bench.py launches them
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("name,n_sample", [("C2", 96), ("C3", 48), ("C4", 40), ("C5", 40)])
+def test_full_size_workloads(name, n_sample):
+    shape = synthetic.CONFIGS[name]
+    inp = inputs_for(shape)
+    run = GpuRun(shape, inp)
+    o = oracle.Oracle(shape, inp)
+    report = {}
+    route = o.forward(route_only=True)                       # norm + router on every token
+    allt = np.arange(shape.T, dtype=np.int32)
+    check_norm(run, route, allt, report)
+    check_routing(run, route, allt, report)
+    toks = sample_tokens(run, route, n_sample, seed=shape.seed)
+    ref = o.forward(toks)
+    check_out(run, ref, toks, report)
+    report["sampled_tokens"] = int(len(toks))
+    report["empty_experts"] = int((run.counts == 0).sum())
+    print(name, json.dumps(report))
+    if name == "C5":
+        assert report["empty_experts"] >= 15
