@@ -28,7 +28,9 @@
  *   - mean(s^2): the exact sum of the squares rounded to double, divided by d in double,
  *     rounded to float32.  rsqrt = 1 / sqrt with IEEE float32 sqrt and divide.
  *   - Linear outputs are in x's dtype (bf16): the expert excerpt's .float() casts imply it.
- *     g = bf16(W1 a), u = bf16(W3 a), h = bf16(silu(g) * u), y_e = bf16(W2 h); sums in float64.
+ *     g = bf16(W1 a), u = bf16(W3 a), y_e = bf16(W2 h); the sums themselves in float64.
+ *     h = bf16(fp32(silu(g)) * fp32(u)): the excerpt fixes float32 for silu and the product;
+ *     silu is taken correctly rounded to float32.
  *   - FP8 activations (performance mode): per token and per 128-column group,
  *     sc = amax / 448 (float32 divide), q = e4m3(v / sc) (float32 divide, round to nearest
  *     even, saturate to +-448); a = q * sc.  amax == 0 gives sc = 1, q = 0.  The same quant
@@ -302,7 +304,11 @@ void oracle_swiglu(int d, int I, int fp8, int act_fp8, const double* a,
         }
         double g = oracle_bf16_to_f64(oracle_f64_to_bf16(gs));   /* w1(x) in x's dtype */
         double u = oracle_bf16_to_f64(oracle_f64_to_bf16(us));   /* w3(x) in x's dtype */
-        h[o] = oracle_bf16_to_f64(oracle_f64_to_bf16(silu(g) * u)); /* .type_as(x) */
+        /* silu(g.float()) * u.float() is float32 arithmetic on the page: silu correctly rounded
+         * to float32, an IEEE float32 multiply, then .type_as(x) */
+        float sg = (float)silu(g);
+        float hv = sg * (float)u;
+        h[o] = oracle_bf16_to_f64(oracle_f64_to_bf16((double)hv));
     }
     if (act_fp8) oracle_act_quant(I, h, NULL, NULL, hq);
     else memcpy(hq, h, sizeof(double) * I);

@@ -9,6 +9,11 @@ Criteria (per workload):
   counts                equal to the bincount of the GPU's own indices
   routing weights       <= 1e-5 relative
   out                   max |err| <= 2e-2 * RMS(oracle out) over the checked elements
+
+Why the layers checked here are not smaller than d = inter = 1024: both sides round g, u and h to
+bf16 and h to e4m3 codes; where float32 accumulation noise lands an intermediate on the other side
+of a rounding midpoint (a legitimate difference), a moved e4m3 code shifts the output by about
+(1/16)/sqrt(inter) of its RMS -- a few percent at inter = 256, well under 1% at 1024 and above.
 """
 from __future__ import annotations
 
@@ -124,16 +129,21 @@ def check_norm(run: GpuRun, ref: dict, tokens: np.ndarray, report: dict):
 
 
 def check_out(run: GpuRun, ref: dict, tokens: np.ndarray, report: dict):
+    """max |err| <= 2e-2 * RMS(oracle out) over the checked elements."""
     g = bf16_bits_to_f64(run.out[tokens])
     o = bf16_bits_to_f64(ref["out"])
     rms = float(np.sqrt(np.mean(o ** 2)))
-    err = float(np.abs(g - o).max())
+    err = np.abs(g - o)
     report["out_rms"] = rms
-    report["out_max_err"] = err
-    report["out_max_err_over_rms"] = err / rms
+    report["out_max_err_over_rms"] = float(err.max() / rms)
     report["out_bitexact_frac"] = float(np.mean(run.out[tokens] == ref["out"]))
     assert np.all(np.isfinite(g))
-    assert err <= OUT_TOL * rms, f"max|err| {err} > {OUT_TOL} * RMS {rms}"
+    tok_err = err.max(1) / rms
+    worst = np.argsort(-tok_err)[:5]
+    diag = [(int(tokens[i]), round(float(tok_err[i]), 4), round(float(np.mean(run.out[tokens[i]] == ref["out"][i])), 4))
+            for i in worst]
+    assert err.max() <= OUT_TOL * rms, \
+        f"max|err|/RMS {err.max() / rms:.4f} > {OUT_TOL} (worst tokens: id, err/RMS, bit-exact fraction: {diag})"
 
 
 def sample_tokens(run: GpuRun, ref_route: dict, n_random: int, seed: int = 0) -> np.ndarray:

@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _shape(**kw):
-    base = dict(name="t", T=300, d=512, I=256, E=16, k=4, n_shared=1, shared_inter=256, wtype="fp8", seed=21)
+    base = dict(name="t", T=300, d=1024, I=1024, E=16, k=4, n_shared=1, shared_inter=1024, wtype="fp8", seed=21)
     base.update(kw)
     return synthetic.MoEShape(**base)
 
@@ -51,7 +51,7 @@ def test_tiny_layer_every_token():
 
 @pytest.mark.parametrize("wtype,T", [("fp8", 300), ("bf16", 200), ("fp8", 1), ("bf16", 129)])
 def test_ragged_layers_every_token(wtype, T):
-    shape = _shape(wtype=wtype, T=T, I=384 if wtype == "bf16" else 256)
+    shape = _shape(wtype=wtype, T=T, I=1152 if wtype == "bf16" else 1024)
     _full_check(shape, inputs_for(shape), {})
 
 
@@ -115,7 +115,7 @@ def test_workspace_and_argument_errors():
     inp = inputs_for(shape)
     cfg = moe.Config.from_shape(shape)
     layer = moe.MoELayer(cfg, {n: v for n, v in inp.items() if n not in ("x", "residual")})
-    out = torch.empty(64, 512, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(64, 1024, dtype=torch.bfloat16, device="cuda")
     ro = torch.empty_like(out)
     small = layer.workspace[: layer.workspace.numel() - 1024]
     rc = moe.moe_forward(cfg, inp["x"], inp["residual"], layer.t["norm_w"], layer.t["gate_w"], None, layer.wstruct,

@@ -228,10 +228,11 @@ def _rb(v):  # round to bf16 and back (torch's cast)
 
 
 def _textbook_swiglu(a, w1, w3, w2):
-    """w2(silu(w1 a) * w3 a), with the Linear outputs rounded to bf16 as the expert excerpt implies."""
+    """w2(silu(w1 a) * w3 a), with the Linear outputs rounded to bf16 as the expert excerpt implies and
+    silu * mul in float32 (silu correctly rounded to float32, float32 product)."""
     g = _rb(w1 @ a)
     u = _rb(w3 @ a)
-    h = _rb(torch.nn.functional.silu(g) * u)
+    h = (torch.nn.functional.silu(g).float() * u.float()).to(torch.bfloat16).double()
     return _rb(w2 @ h)
 
 
