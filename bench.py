@@ -178,7 +178,8 @@ def run_reference(args, shape, rank):
 
 
 def config_block(shape):
-    return {"workload": f"{shape.name}: {synthetic.DESCRIPTIONS[shape.name]}", "tokens": shape.T, "dim": shape.d,
+    desc = synthetic.DESCRIPTIONS.get(shape.name, "reduced case of " + shape.name.split("-")[0] + " (profiling only)")
+    return {"workload": f"{shape.name}: {desc}", "tokens": shape.T, "dim": shape.d,
             "moe_inter": shape.I, "experts": shape.E, "top_k": shape.k, "shared_inter": shape.Is,
             "weights": "e4m3 + fp32 128x128 block scales" if shape.wtype == "fp8" else "bf16",
             "activations": "e4m3 1x128 groups into the expert GEMMs" if shape.wtype == "fp8" else "bf16",
@@ -298,7 +299,7 @@ def run_ours(args, shape, rank, world, device):
                           "gbs_frac_of_hbm": wk["step_bytes"] / (ms * 1e-3) / 1e9 / P["hbm_gbs"],
                           "touched_experts": wk["touched"]},
         "stage_ms": {n: float(stage[:, j].mean()) for j, n in enumerate(
-            ["norm", "gate_gemm", "topk_recheck", "route", "gemm_up", "gemm_down", "combine"])},
+            ["norm", "gate_gemm", "topk", "route", "gemm_up", "gemm_down", "combine"])},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": 2 * x.numel() * 2,
                 "d2h_bytes_per_step": 2 * x.numel() * 2, "ms_per_step": e2e_ms},
         "gpu_launches": moe.launches_per_forward(cfg) * K,
@@ -318,9 +319,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--tokens", type=int, default=0, help="override T (smaller cases for profiling)")
+    ap.add_argument("--experts", type=int, default=0, help="override E (smaller cases for profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     shape = synthetic.CONFIGS[args.config]
+    if args.tokens or args.experts:
+        shape = dataclasses.replace(shape, name=shape.name + "-reduced", T=args.tokens or shape.T,
+                                    E=args.experts or shape.E, zipf_bias=False)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -19,9 +19,10 @@
  *     block, scale shape [ceil(out/128), ceil(in/128)].
  *
  * The router's body is not on the pages.  This library computes scores = sigmoid(xn . Wg_e +
- * bias_e) in float32, keeps the top_k experts (on equal scores the lower expert index wins),
- * normalises their scores to sum 1, and re-decides in float64 every token whose k-th and
- * (k+1)-th float32 scores are closer than tie_tau.
+ * bias_e), keeps the top_k experts (on equal scores the lower expert index wins) and normalises
+ * their scores to sum 1.  Logits come from a float32 tensor-core GEMM; the winners and every
+ * expert within 2e-3 (logit units) of the k-th winner are re-evaluated in float64, so the
+ * selection is the exact one and the weights are float64 scores rounded to float32.
  *
  * Conventions for every entry point
  *   - Tensors are device pointers (CUDA global memory of the current device), contiguous and
@@ -81,8 +82,6 @@ typedef struct {
     int32_t wtype;         /* moe_wtype_t, same for routed and shared weights */
     int32_t amode;         /* moe_amode_t; FP8 weights need MOE_ACT_FP8_1x128 in this build */
     float eps;             /* RMSNorm eps (1e-6 on the pages) */
-    float tie_tau;         /* float32 score margin below which a token is re-routed in float64;
-                              <= 0 selects the default 1e-4 */
 } moe_config_t;
 
 /* Expert weights, [out, in] row-major.  Routed: w1, w3 [E, I, d]; w2 [E, d, I].
@@ -124,7 +123,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* res
  *   events[0] before the first launch      events[4] after the permutation kernels
  *   events[1] after the norm kernel        events[5] after the grouped GEMM up (w1|w3, SwiGLU)
  *   events[2] after the gate GEMM          events[6] after the grouped GEMM down (w2)
- *   events[3] after top-k + recheck        events[7] after the combine kernel
+ *   events[3] after the top-k kernel       events[7] after the combine kernel
  * n_events may be smaller than 8 (the later boundaries are then not recorded); NULL entries are
  * skipped.  Same arguments, errors and ownership as moe_forward otherwise. */
 moe_status_t moe_forward_traced(const moe_config_t* cfg, const void* x, const void* residual,
@@ -134,13 +133,16 @@ moe_status_t moe_forward_traced(const moe_config_t* cfg, const void* x, const vo
                                 void* const* events, int32_t n_events);
 
 /* Synchronises `stream`, then returns the status latched in the workspace by the last
- * moe_forward on it (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_CHECK), or MOE_ERR_CUDA. */
+ * moe_forward on it (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or MOE_ERR_DEVICE_CHECK), or MOE_ERR_CUDA.
+ * Undefined for a workspace no moe_forward has run on yet (the call that clears the status word
+ * is the first thing moe_forward enqueues). */
 moe_status_t moe_get_status(const void* workspace, void* stream);
 
 /* Copies (device to device, enqueued on `stream`) the routing of the last moe_forward that
  * used this workspace: idx [T, k] int32 (slot order = descending score), weights [T, k]
- * float32, counts [E] int32 (tokens per expert), near_tie [T] uint8 (1 = the token was
- * re-decided in float64).  Any output pointer may be NULL. */
+ * float32, counts [E] int32 (tokens per expert), near_tie [T] uint8 (1 = another expert was
+ * within the candidate window of the k-th winner and the selection was re-decided in float64).
+ * Any output pointer may be NULL. */
 moe_status_t moe_debug_routing(const moe_config_t* cfg, const void* workspace, int32_t* idx,
                                float* weights, int32_t* counts, uint8_t* near_tie, void* stream);
 

@@ -32,7 +32,7 @@ class MoeError(RuntimeError):
 class moe_config_t(C.Structure):
     _fields_ = [("num_tokens", C.c_int32), ("dim", C.c_int32), ("inter_dim", C.c_int32), ("n_experts", C.c_int32),
                 ("top_k", C.c_int32), ("shared_inter", C.c_int32), ("wtype", C.c_int32), ("amode", C.c_int32),
-                ("eps", C.c_float), ("tie_tau", C.c_float)]
+                ("eps", C.c_float)]
 
 
 class moe_weights_t(C.Structure):
@@ -86,18 +86,17 @@ class Config:
     wtype: int = MOE_W_FP8_E4M3_B128
     amode: int = MOE_ACT_FP8_1x128
     eps: float = 1e-6
-    tie_tau: float = 0.0
 
     def c(self) -> moe_config_t:
         return moe_config_t(self.num_tokens, self.dim, self.inter_dim, self.n_experts, self.top_k, self.shared_inter,
-                            self.wtype, self.amode, self.eps, self.tie_tau)
+                            self.wtype, self.amode, self.eps)
 
     @staticmethod
-    def from_shape(shape, num_tokens=None, tie_tau=0.0) -> "Config":
+    def from_shape(shape, num_tokens=None) -> "Config":
         fp8 = shape.wtype == "fp8"
         return Config(num_tokens or shape.T, shape.d, shape.I, shape.E, shape.k, shape.Is,
                       MOE_W_FP8_E4M3_B128 if fp8 else MOE_W_BF16, MOE_ACT_FP8_1x128 if fp8 else MOE_ACT_BF16,
-                      shape.eps, tie_tau)
+                      shape.eps)
 
 
 def _ptr(t):

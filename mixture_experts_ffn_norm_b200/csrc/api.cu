@@ -2,7 +2,7 @@
 // sequence of one forward pass.  Nothing here waits on the device except moe_get_status.
 //
 // Launch sequence (one stream, no host sync; every routing-dependent size is read on the device):
-//   norm -> gate GEMM (logits) -> top-k -> float64 near-tie recheck -> hist -> scan -> scatter
+//   norm -> gate GEMM (logits) -> top-k with float64 re-decision -> hist -> scan -> scatter
 //   -> gather -> grouped GEMM up (w1|w3 + SwiGLU) -> grouped GEMM down (w2) -> combine
 #include <algorithm>
 #include <cstring>
@@ -96,7 +96,6 @@ bool make_layout(const moe_config_t& c, Layout& L) {
     L.idx = take(static_cast<size_t>(L.T) * L.k * 4);
     L.w = take(static_cast<size_t>(L.T) * L.k * 4);
     L.flag = take(L.T);
-    L.flag_list = take(static_cast<size_t>(L.T) * 4);
     L.counts = take(static_cast<size_t>(L.E) * 4);
     L.offsets = take(static_cast<size_t>(L.E + 1) * 4);
     L.row_base = take(static_cast<size_t>(L.E + 1) * 4);
@@ -147,7 +146,7 @@ extern "C" size_t moe_workspace_bytes(const moe_config_t* cfg) {
 extern "C" int32_t moe_launches_per_forward(const moe_config_t* cfg) {
     Layout L;
     if (check_config(cfg, L) != MOE_OK) return 0;
-    return 11;   // norm, gate GEMM, top-k, recheck, hist, scan, scatter, gather, up, down, combine
+    return 10;   // norm, gate GEMM, top-k, hist, scan, scatter, gather, up, down, combine
 }
 
 static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const void* residual,
@@ -180,7 +179,6 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
                                                      : cudaSuccess;
     };
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    const float tau = cfg->tie_tau > 0.0f ? cfg->tie_tau : 1e-4f;
     const int sms = num_sms();
     const bool fp8 = L.fp8;
 
@@ -214,9 +212,8 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
         MOE_TRY(launch_gemm(kModeLogits, false, m, p, std::min(tiles, sms), s));
     }
     MOE_TRY(mark(2));
-    // 3. top-k + float64 recheck of near ties
-    MOE_TRY(launch_topk(L, gate_bias, tau, ws, s));
-    MOE_TRY(launch_recheck(L, gate_w, gate_bias, ws, s));
+    // 3. top-k, re-decided in float64 near the boundary
+    MOE_TRY(launch_topk(L, gate_w, gate_bias, ws, s));
     MOE_TRY(mark(3));
 
     // 4. permutation by expert

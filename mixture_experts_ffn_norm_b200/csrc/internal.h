@@ -25,7 +25,7 @@ enum GemmMode : int { kModeLogits = 0, kModeUp = 1, kModeDown = 2 };
 struct Layout {
     int T, d, I, E, k, Is, Tpad, R, KBd, KBi, KBs, nchunks;
     bool fp8, act8;
-    size_t status, xn, xq, xs, logits, idx, w, flag, flag_list, counts, offsets, row_base, row_count,
+    size_t status, xn, xq, xs, logits, idx, w, flag, counts, offsets, row_base, row_count,
         ts_up, ts_down, chunk_hist, row_of, row_token, a_perm, as_perm, h, hs, h_sh, hs_sh, y, y_sh, total;
 };
 
@@ -71,9 +71,7 @@ cudaError_t launch_norm(const Layout& L, const void* x, const void* residual, co
                         void* residual_out, uint8_t* ws, cudaStream_t s);
 cudaError_t launch_gemm(int mode, bool fp8, const TensorMaps& maps, const GemmParams& p, int grid,
                         cudaStream_t s);
-cudaError_t launch_topk(const Layout& L, const float* gate_bias, float tau, uint8_t* ws, cudaStream_t s);
-cudaError_t launch_recheck(const Layout& L, const void* gate_w, const float* gate_bias, uint8_t* ws,
-                           cudaStream_t s);
+cudaError_t launch_topk(const Layout& L, const void* gate_w, const float* gate_bias, uint8_t* ws, cudaStream_t s);
 cudaError_t launch_route(const Layout& L, int ntu_r, int ntu_s, int ntd_r, int ntd_s, uint8_t* ws,
                          cudaStream_t s);
 cudaError_t launch_combine(const Layout& L, void* out, uint8_t* ws, cudaStream_t s);

@@ -9,7 +9,7 @@
 namespace moe {
 
 // status word layout (uint32 words at the start of the workspace)
-enum : int { kStatusErr = 0, kStatusWhere = 1, kStatusFlagCount = 2, kStatusWords = 64 };
+enum : int { kStatusErr = 0, kStatusWhere = 1, kStatusWords = 64 };
 enum : uint32_t { kErrTimeout = 5u, kErrCheck = 6u };
 
 // ~2^31 cycles: about a second at the B200's clocks; no legitimate wait is near this.

@@ -54,9 +54,9 @@ def bits_np(t: torch.Tensor) -> np.ndarray:
 class GpuRun:
     """One moe_forward through the C ABI plus every debug export, copied to the host."""
 
-    def __init__(self, shape, inp: dict, residual=True, in_place=False, tie_tau=0.0, cfg=None):
+    def __init__(self, shape, inp: dict, residual=True, in_place=False, cfg=None):
         self.shape = shape
-        self.cfg = cfg or moe.Config.from_shape(shape, tie_tau=tie_tau)
+        self.cfg = cfg or moe.Config.from_shape(shape)
         dev = inp["x"].device
         T, d, k, E = self.cfg.num_tokens, self.cfg.dim, self.cfg.top_k, self.cfg.n_experts
         self.layer = moe.MoELayer(self.cfg, {n: v for n, v in inp.items() if n not in ("x", "residual")}, device=dev)
@@ -128,8 +128,19 @@ def check_norm(run: GpuRun, ref: dict, tokens: np.ndarray, report: dict):
             assert np.array_equal(run.xs[:, t], sc), f"xs differs for token {t}"
 
 
-def check_out(run: GpuRun, ref: dict, tokens: np.ndarray, report: dict):
-    """max |err| <= 2e-2 * RMS(oracle out) over the checked elements."""
+def ulp_bf16(v):
+    a = np.maximum(np.abs(np.asarray(v, np.float64)), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+def check_out(run: GpuRun, ref: dict, tokens: np.ndarray, report: dict, allow_ulp: bool = False):
+    """max |err| <= 2e-2 * RMS(oracle out) over the checked elements.
+
+    allow_ulp (used only by the structural edge-case layers, never by the five workloads): an
+    element may also differ by one bf16 step of the oracle's value.  Both sides round g, u, h and
+    every expert output to bf16; where float32 accumulation lands one of them on the other side of
+    a midpoint, the token's outputs move by a fraction of a step and some round one step apart --
+    and one step of an element beyond ~3 sigma is already more than 2e-2 * RMS."""
     g = bf16_bits_to_f64(run.out[tokens])
     o = bf16_bits_to_f64(ref["out"])
     rms = float(np.sqrt(np.mean(o ** 2)))
@@ -142,7 +153,11 @@ def check_out(run: GpuRun, ref: dict, tokens: np.ndarray, report: dict):
     worst = np.argsort(-tok_err)[:5]
     diag = [(int(tokens[i]), round(float(tok_err[i]), 4), round(float(np.mean(run.out[tokens[i]] == ref["out"][i])), 4))
             for i in worst]
-    assert err.max() <= OUT_TOL * rms, \
+    tol = OUT_TOL * rms
+    if allow_ulp:
+        tol = np.maximum(tol, ulp_bf16(o) * (1 + 1e-12))
+        report["out_beyond_2e-2_rms_within_1ulp"] = int((err > OUT_TOL * rms).sum())
+    assert np.all(err <= tol), \
         f"max|err|/RMS {err.max() / rms:.4f} > {OUT_TOL} (worst tokens: id, err/RMS, bit-exact fraction: {diag})"
 
 
