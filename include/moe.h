@@ -152,6 +152,33 @@ moe_status_t moe_debug_routing(const moe_config_t* cfg, const void* workspace, i
 moe_status_t moe_debug_norm(const moe_config_t* cfg, const void* workspace, void* xn,
                             void* xq, float* xs, void* stream);
 
+/* The expert grouping step alone -- tokens per expert, expert offsets and the permutation by
+ * expert -- computed exactly as moe_forward computes it internally, but without any workspace.
+ * The pages have no counterpart: this entry point exists for callers that cannot allocate
+ * device memory when they call in, e.g. a serving runtime that reserves all device memory up
+ * front and hands a layer only the tensors it reads and writes, or code on a latency-critical
+ * path where a cudaMalloc would synchronise the device and stall every other stream.
+ *   idx        [T, k] int32 device      expert of every (token, slot); values in [0, E)
+ *   counts     [E] int32 device         tokens routed to each expert
+ *   offsets    [E + 1] int32 device     first permuted row of each expert; each expert's rows
+ *                                       start on a multiple of 128; offsets[E] = rows used
+ *   row_of     [T, k] int32 device      permuted row of every (token, slot); inside an expert
+ *                                       the rows follow token order
+ *   row_token  [R] int32 device         token of every permuted row, -1 in padding rows, with
+ *                                       R = roundup(T*k + 127*E, 128)
+ * Its scratch (per-chunk histograms and tables, 136 KiB) is one file-scope device array that
+ * every device loading the library holds until the process exits.  T*k may be at most 262144;
+ * larger sizes return MOE_ERR_UNSUPPORTED.  The first call on a device looks up the array's
+ * device address with that device current (the caller's current device must own `stream`), so
+ * make that first call before any stream capture.  Calls share the array: two calls whose work
+ * overlaps on the GPU (different streams, or different host threads) race and give wrong
+ * results; calls ordered on one stream are fine.  Nothing left in the array by an earlier call
+ * is read.  No allocation of any kind is made.  Errors: MOE_ERR_INVALID_ARG for NULL pointers
+ * or sizes out of range, MOE_ERR_CUDA for a failed lookup or launch. */
+moe_status_t moe_route_noalloc(const int32_t* idx, int32_t num_tokens, int32_t top_k, int32_t n_experts,
+                               int32_t* counts, int32_t* offsets, int32_t* row_of, int32_t* row_token,
+                               void* stream);
+
 /* Number of kernel launches one moe_forward enqueues for this configuration. */
 int32_t moe_launches_per_forward(const moe_config_t* cfg);
 

@@ -19,8 +19,8 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
 MOE_W_BF16, MOE_W_FP8_E4M3_B128 = 0, 1
 MOE_ACT_FP8_1x128, MOE_ACT_BF16 = 0, 1
 
-EXPORTS = ("moe_workspace_bytes", "moe_forward", "moe_forward_traced", "moe_get_status", "moe_debug_routing", "moe_debug_norm",
-           "moe_launches_per_forward", "moe_status_string")
+EXPORTS = ("moe_workspace_bytes", "moe_forward", "moe_forward_traced", "moe_get_status", "moe_debug_routing",
+           "moe_debug_norm", "moe_route_noalloc", "moe_launches_per_forward", "moe_status_string")
 
 
 class MoeError(RuntimeError):
@@ -63,6 +63,8 @@ def lib() -> C.CDLL:
         L.moe_debug_routing.argtypes = [cfgp, vp, vp, vp, vp, vp, vp]
         L.moe_debug_norm.restype = C.c_int
         L.moe_debug_norm.argtypes = [cfgp, vp, vp, vp, vp, vp]
+        L.moe_route_noalloc.restype = C.c_int
+        L.moe_route_noalloc.argtypes = [vp, C.c_int32, C.c_int32, C.c_int32, vp, vp, vp, vp, vp]
         L.moe_launches_per_forward.restype = C.c_int32
         L.moe_launches_per_forward.argtypes = [cfgp]
         L.moe_status_string.restype = C.c_char_p
@@ -164,6 +166,22 @@ def moe_debug_norm(cfg: Config, workspace, xn=None, xq=None, xs=None, stream=Non
     rc = lib().moe_debug_norm(C.byref(cfg.c()), _ptr(workspace), _ptr(xn), _ptr(xq), _ptr(xs), _stream(stream))
     if rc != MOE_OK:
         raise MoeError(rc, "moe_debug_norm")
+
+
+def route_rows(num_tokens: int, top_k: int, n_experts: int) -> int:
+    """Capacity R of the permuted-row space: roundup(T*k + 127*E, 128)."""
+    return (num_tokens * top_k + 127 * n_experts + 127) // 128 * 128
+
+
+def moe_route_noalloc(idx, n_experts: int, counts, offsets, row_of, row_token, stream=None, check=True) -> int:
+    """Expert grouping without any workspace (see moe_route_noalloc in include/moe.h).  idx: [T, k]
+    int32 device tensor; outputs are caller-provided int32 device tensors."""
+    T, k = idx.shape
+    rc = lib().moe_route_noalloc(_ptr(idx), T, k, n_experts, _ptr(counts), _ptr(offsets), _ptr(row_of),
+                                 _ptr(row_token), _stream(stream))
+    if check and rc != MOE_OK:
+        raise MoeError(rc, "moe_route_noalloc")
+    return rc
 
 
 class MoELayer:

@@ -10,6 +10,8 @@
 //             so the permutation is deterministic);
 //   gather  : the permuted activation rows (FP8 codes or bf16) and their group scales are
 //             copied next to each other so a TMA box of 128 rows is one expert's tile.
+#include <mutex>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -178,4 +180,75 @@ cudaError_t launch_route(const Layout& L, int ntu_r, int ntu_s, int ntd_r, int n
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------------------------------
+// moe_route_noalloc: the same counting / scan / permutation, for callers that cannot allocate.
+//
+// Its scratch -- the per-chunk histograms and the tile tables the scan also produces -- lives in
+// one file-scope device array instead of a caller workspace.  The array exists once per device
+// for the life of the process; every call on a device shares it.
+// ------------------------------------------------------------------------------------------------
+namespace {
+
+constexpr int kNoAllocMaxEntries = 1 << 18;                               // T * k
+constexpr int kNoAllocMaxChunks = kNoAllocMaxEntries / kRouteChunk;       // 128
+constexpr int kNoAllocHist = kNoAllocMaxChunks * kMaxExperts;             // ints
+constexpr int kNoAllocTables = 2 * (kMaxExperts + 1) + 2 * (kMaxExperts + 2);
+constexpr int kNoAllocInts = kNoAllocHist + kNoAllocTables;                // 34,818 ints = 136 KiB
+
+static __device__ __align__(256) int g_route_scratch[kNoAllocInts];
+
+constexpr int kMaxDevices = 64;
+int* g_scratch_ptr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// Device address of g_route_scratch on the current device, looked up once per device.  In host
+// code the array's name is only a host-side stand-in, so it must never be passed to a kernel.
+cudaError_t scratch_for_current_device(int** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_route_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = static_cast<int*>(p);
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
 }  // namespace moe
+
+extern "C" moe_status_t moe_route_noalloc(const int32_t* idx, int32_t num_tokens, int32_t top_k, int32_t n_experts,
+                                          int32_t* counts, int32_t* offsets, int32_t* row_of, int32_t* row_token,
+                                          void* stream) {
+    using namespace moe;
+    if (!idx || !counts || !offsets || !row_of || !row_token) return MOE_ERR_INVALID_ARG;
+    if (num_tokens < 1 || top_k < 1 || n_experts < 1 || n_experts > kMaxExperts || top_k > n_experts)
+        return MOE_ERR_INVALID_ARG;
+    const long long n = static_cast<long long>(num_tokens) * top_k;
+    if (n > kNoAllocMaxEntries) return MOE_ERR_UNSUPPORTED;   // beyond the static scratch
+    int* scratch = nullptr;
+    if (scratch_for_current_device(&scratch) != cudaSuccess) return MOE_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int N = static_cast<int>(n), E = n_experts;
+    const int nchunks = (N + kRouteChunk - 1) / kRouteChunk;
+    const long long rows = (n + static_cast<long long>(E) * (kBM - 1) + kBM - 1) / kBM * kBM;
+    int* hist = scratch;
+    int* row_base = scratch + kNoAllocHist;
+    int* row_count = row_base + (kMaxExperts + 1);
+    int* ts_up = row_count + (kMaxExperts + 1);
+    int* ts_down = ts_up + (kMaxExperts + 2);
+    // every histogram entry the scan reads is written by hist_kernel first, so nothing left in
+    // the array by an earlier call is read; row_token's padding must read -1
+    if (cudaMemsetAsync(row_token, 0xFF, static_cast<size_t>(rows) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+    hist_kernel<<<nchunks, kRouteThreads, 0, s>>>(idx, N, E, hist, nullptr);
+    scan_kernel<<<1, kRouteThreads, 0, s>>>(hist, nchunks, E, num_tokens, 0, 1, 1, 1, 1, counts, offsets, row_base,
+                                            row_count, ts_up, ts_down);
+    scatter_kernel<<<nchunks, kRouteThreads, 0, s>>>(idx, N, E, top_k, hist, offsets, row_of, row_token);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
