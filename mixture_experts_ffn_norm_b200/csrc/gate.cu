@@ -5,12 +5,13 @@
 // scores, and the winners' scores are normalised to sum 1.
 //
 // One warp per token.  The E <= 256 float32 logits (+ bias) are spread over the lanes and the
-// top k are picked by k rounds of a warp-wide (value, lower index) argmax.  The tensor core's
-// float32 logits carry an absolute error of a few 1e-5, so the set S = {the k winners} U {every
-// other expert within kCandDelta of the k-th winner} is then re-evaluated in float64 (bf16 x bf16
-// products are exact in float64): every expert outside S is provably below all k winners, so
-// re-deciding the top k inside S in float64 gives the exact selection, and the weights come from
-// float64 scores.  A token with any candidate besides its winners is marked as re-decided.
+// top k are picked by k rounds of a warp-wide (value, lower index) argmax.  The logits GEMM
+// promotes every 64-wide K stage into float32 registers, so a logit is off by ~1e-6; kCandDelta
+// is far above that.  When another expert lies within kCandDelta of the k-th winner, the set
+// S = {winners} U {those candidates} is re-evaluated in float64 (bf16 x bf16 products are exact in
+// float64) and the top k is re-decided inside S: every expert outside S is provably below all k
+// winners, so the selection is the exact one.  Such tokens are marked as re-decided and their
+// weights come from float64 scores; the others take float64 sigmoids of their float32 logits.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -23,7 +24,7 @@ namespace moe {
 namespace {
 
 constexpr int kTopkWarps = 8;
-constexpr float kCandDelta = 2e-3f;   // logit units; ~40x the largest float32 logit error observed
+constexpr float kCandDelta = 2e-3f;   // logit units; far above the float32 logit error
 
 __device__ __forceinline__ bool better(float za, int ea, float zb, int eb) {
     return za > zb || (za == zb && ea < eb);
@@ -105,27 +106,27 @@ topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, co
         if (((valid & ~taken) >> j) & 1u && z[j] >= zk - kCandDelta) cand |= 1u << j;
     const bool redo = __any_sync(0xFFFFFFFFu, cand != 0);
     const uint32_t S = taken | cand;
-    // float64 scores of every member of S (each lane keeps its own experts' values)
-    const int nv = d >> 3;
-    const uint4* xr = reinterpret_cast<const uint4*>(xn + static_cast<size_t>(t) * d);
     double s64[J];
-#pragma unroll
-    for (int j = 0; j < J; ++j) {
-        s64[j] = -1.0;
-        uint32_t m = __ballot_sync(0xFFFFFFFFu, (S >> j) & 1u);
-        while (m) {
-            const int src = __ffs(m) - 1;
-            m &= m - 1;
-            const int e = src + 32 * j;
-            double zz = dot64(xr, reinterpret_cast<const uint4*>(gw + static_cast<size_t>(e) * d), nv, lane);
-            if (bias) zz += static_cast<double>(bias[e]);
-            if (lane == src) s64[j] = 1.0 / (1.0 + exp(-zz));
-        }
-    }
-    // the final k: re-decided inside S by float64 score (lower index first on ties) when candidates
-    // exist, else the float32 winners (the same set)
-    uint32_t fin = redo ? 0u : taken;
+    uint32_t fin = taken;
     if (redo) {
+        // float64 scores of every member of S (each lane keeps its own experts' values), then the
+        // top k inside S by float64 score, lower index first on equal scores
+        const int nv = d >> 3;
+        const uint4* xr = reinterpret_cast<const uint4*>(xn + static_cast<size_t>(t) * d);
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            s64[j] = -1.0;
+            uint32_t m = __ballot_sync(0xFFFFFFFFu, (S >> j) & 1u);
+            while (m) {
+                const int src = __ffs(m) - 1;
+                m &= m - 1;
+                const int e = src + 32 * j;
+                double zz = dot64(xr, reinterpret_cast<const uint4*>(gw + static_cast<size_t>(e) * d), nv, lane);
+                if (bias) zz += static_cast<double>(bias[e]);
+                if (lane == src) s64[j] = 1.0 / (1.0 + exp(-zz));
+            }
+        }
+        fin = 0u;
         for (int rnd = 0; rnd < k; ++rnd) {
             double bs = -2.0;
             int be = 0x7FFFFFFF;
@@ -148,8 +149,13 @@ topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, co
             }
             if ((be & 31) == lane) fin |= 1u << (be >> 5);
         }
+    } else {
+        // no expert near the boundary: the float32 winners are the top k; scores from the float32
+        // logits (promoted per 64-wide K stage, so their error is ~1e-6)
+#pragma unroll
+        for (int j = 0; j < J; ++j) s64[j] = ((taken >> j) & 1u) ? 1.0 / (1.0 + exp(-static_cast<double>(z[j]))) : 0.0;
     }
-    // weights = float64 scores / their sum; slots in ascending expert order
+    // weights = scores / their sum; slots in ascending expert order
     double sum = 0.0;
 #pragma unroll
     for (int j = 0; j < J; ++j)

@@ -15,10 +15,15 @@
 // registers.  Two TMEM buffers (2 x 256 columns) let the MMA of block kb+1 run while block kb is
 // promoted.  bf16 operands simply accumulate the whole K in TMEM.
 //
-// Warp roles (320 threads, one CTA per SM, persistent over a device-side tile table):
+// Warp roles (384 threads = 3 warpgroups, one CTA per SM, persistent over a device-side tile table):
 //   warp 0      one thread issues the TMA loads of A (128 x 128 B) and B (256 x 128 B) per stage
 //   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=32 bytes per instruction)
-//   warps 2..9  epilogue: warp w reads TMEM lanes 32*(w%4).., column half (w-2)/4
+//   warps 2-3   idle (they only hand their registers back)
+//   warps 4..11 epilogue: warp w reads TMEM lanes 32*(w%4).., column half (w-4)/4
+// setmaxnreg moves registers from warpgroup 0 (56 each) to the two epilogue warpgroups (224 each):
+// 128*56 + 256*224 = 64512 = 384 * 168, the launch budget.  The FP8 promotion keeps 128 float32
+// accumulators per thread, loads 64 TMEM columns per wait, accumulates with packed fp32x2 FMAs and
+// prefetches the next K block's scales while it waits.
 // Tiles are taken m-fastest inside a group so concurrently running CTAs share the weight tile
 // through L2.  Every wait is bounded (see ptx.cuh); on a timeout all roles leave their loops,
 // in-flight TMA loads and MMAs are drained with bounded waits, and TMEM is freed.
@@ -143,7 +148,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
     const uint32_t tmem = tmem_base_sh;
     const int total = ts_sh[p.G];
 
-    if (warp == 0) {
+    if (warp < 4) {
+      regs_dec<56>();
+      if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tensormap(&tm_a_r);
@@ -190,6 +197,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = instr_desc(kFp8, kBM, kBN);
+            constexpr bool kPromote = kFp8 || kMode == kModeLogits;
             int stage = 0, abuf = 0;
             uint32_t phase = 0, aphase = 0;
             bool ok = true;
@@ -197,7 +205,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                 Tile ti;
                 decode_tile(t, ts_sh, rb_sh, rc_sh, p, kMode, ti);
                 for (int kb = 0; kb < ti.kb; ++kb) {
-                    if (kFp8 || kb == 0) {
+                    if (kPromote || kb == 0) {
                         if (!mbar_wait(&tempty_bar[abuf], aphase ^ 1u, &abort_sh, p.status, 0x20)) {
                             ok = false;
                             break;
@@ -215,9 +223,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                     const uint32_t dt = tmem + static_cast<uint32_t>(abuf * kBN);
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        umma<kFp8>(dt, ad + 2 * ks, bd + 2 * ks, idesc, kFp8 ? (ks > 0) : (kb > 0 || ks > 0));
+                        umma<kFp8>(dt, ad + 2 * ks, bd + 2 * ks, idesc, kPromote ? (ks > 0) : (kb > 0 || ks > 0));
                     umma_commit(&empty_bar[stage]);
-                    if (kFp8 || kb == ti.kb - 1) {
+                    if (kPromote || kb == ti.kb - 1) {
                         umma_commit(&tfull_bar[abuf]);
                         abuf ^= 1;
                         if (abuf == 0) aphase ^= 1u;
@@ -231,10 +239,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
             umma_commit(&drain_bar);
             drain_wait(&drain_bar, 0);
         }
+      }
     } else {
+        regs_inc<224>();
         // ------------------------------------------------------------------ epilogue
         const int q = warp & 3;
-        const int c = (warp - 2) >> 2;
+        const int c = (warp - 4) >> 2;
         const int r = q * 32 + lane;
         const uint32_t tl = tmem + (static_cast<uint32_t>(q * 32) << 16);
         int abuf = 0;
@@ -246,52 +256,97 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
             const bool valid = r < ti.rows_valid;
             uint8_t* out = static_cast<uint8_t*>(ti.shared ? p.out_s : p.out_r);
             const size_t out_ld = static_cast<size_t>(ti.shared ? p.out_ld_s : p.out_ld_r);
-            if constexpr (kFp8) {
-                float acc[128];
+            if constexpr (kFp8 || kMode == kModeLogits) {
+                // promotion: every K stage arrives in its own TMEM buffer and is added into float32
+                // registers (FP8: scaled by s_act[row, kb] * s_w[blk, kb]; logits: scale 1)
+                float2 acc[64];
 #pragma unroll
-                for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+                for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.0f, 0.0f);
+                constexpr bool kScaled = kFp8;
                 const float* as = ti.shared ? p.as_s : p.as_r;
                 const size_t as_ld = static_cast<size_t>(ti.shared ? p.as_ld_s : p.as_ld_r);
                 const int bcols = ti.shared ? p.bs_cols_s : p.bs_cols_r;
                 const int brow = (ti.shared ? 0 : ti.g * p.bs_rows_r) + (kMode == kModeUp ? ti.nt : 2 * ti.nt + c);
-                const float* sc0 = (ti.shared ? p.bs0_s : p.bs0_r) + static_cast<size_t>(brow) * bcols;
-                const float* sc1 = (ti.shared ? p.bs1_s : p.bs1_r) + static_cast<size_t>(brow) * bcols;
+                const float* sc0 = kScaled ? (ti.shared ? p.bs0_s : p.bs0_r) + static_cast<size_t>(brow) * bcols : nullptr;
+                const float* sc1 = kScaled ? (ti.shared ? p.bs1_s : p.bs1_r) + static_cast<size_t>(brow) * bcols : nullptr;
+                // scales of K block 0; each iteration fetches the next block's before it waits
+                float sa = 1.0f, w0 = 1.0f, w1 = 1.0f;
+                if constexpr (kScaled) {
+                    sa = as[grow];
+                    w0 = __ldg(sc0);
+                    w1 = (kMode == kModeUp) ? __ldg(sc1) : 0.0f;
+                }
                 bool ok = true;
                 for (int kb = 0; kb < ti.kb; ++kb) {
+                    const int kn = kb + 1 < ti.kb ? kb + 1 : kb;
+                    float sa_n = 1.0f, w0_n = 1.0f, w1_n = 1.0f;
+                    if constexpr (kScaled) {
+                        sa_n = as[static_cast<size_t>(kn) * as_ld + grow];
+                        w0_n = __ldg(sc0 + kn);
+                        w1_n = (kMode == kModeUp) ? __ldg(sc1 + kn) : 0.0f;
+                    }
                     if (!mbar_wait(&tfull_bar[abuf], aphase, &abort_sh, p.status, 0x30)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const float sa = as[static_cast<size_t>(kb) * as_ld + grow];
-                    const float f0 = sa * __ldg(sc0 + kb);
-                    const float f1 = (kMode == kModeUp) ? sa * __ldg(sc1 + kb) : f0;
+                    const float f0 = sa * w0;
+                    const float f1 = (kMode == kModeUp) ? sa * w1 : f0;
+                    const float2 f0v = make_float2(f0, f0), f1v = make_float2(f1, f1);
                     const uint32_t base = tl + static_cast<uint32_t>(abuf * kBN);
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const int col = (kMode == kModeUp) ? ((ch < 2 ? 0 : 128) + 64 * c + 32 * (ch & 1))
-                                                           : (128 * c + 32 * ch);
-                        uint32_t v[32];
-                        tmem_ld32(base + col, v);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        // UP: hh 0 = g columns (64c..), hh 1 = u columns (128+64c..); DOWN: 128c + 64hh
+                        const int col = (kMode == kModeUp) ? (hh ? 128 : 0) + 64 * c : 128 * c + 64 * hh;
+                        uint32_t v0[32], v1[32];
+                        tmem_ld32(base + col, v0);
+                        tmem_ld32(base + col + 32, v1);
                         tmem_wait_ld();
-                        const float f = (ch < 2) ? f0 : f1;
+                        const float2 fv = hh ? f1v : f0v;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) acc[ch * 32 + j] = fmaf(__uint_as_float(v[j]), f, acc[ch * 32 + j]);
+                        for (int j = 0; j < 16; ++j) {
+                            acc[hh * 32 + j] = __ffma2_rn(make_float2(__uint_as_float(v0[2 * j]), __uint_as_float(v0[2 * j + 1])),
+                                                          fv, acc[hh * 32 + j]);
+                            acc[hh * 32 + 16 + j] = __ffma2_rn(
+                                make_float2(__uint_as_float(v1[2 * j]), __uint_as_float(v1[2 * j + 1])), fv,
+                                acc[hh * 32 + 16 + j]);
+                        }
                     }
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&tempty_bar[abuf]);
                     abuf ^= 1;
                     if (abuf == 0) aphase ^= 1u;
+                    sa = sa_n;
+                    w0 = w0_n;
+                    w1 = w1_n;
                 }
                 if (!ok) break;
-                if constexpr (kMode == kModeUp) {
+                float* accf = reinterpret_cast<float*>(acc);
+                if constexpr (kMode == kModeLogits) {
+                    // router logits, float32, columns 128c .. 128c+127 that are < n_valid_cols
+                    if (valid) {
+                        float* dst = reinterpret_cast<float*>(out + static_cast<size_t>(grow) * out_ld * 4) + 128 * c;
+                        const int ncol = min(128, p.n_valid_cols - 128 * c);
+                        if ((p.n_valid_cols & 3) == 0) {        // rows 16-byte aligned: vector stores
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (4 * i < ncol)
+                                    reinterpret_cast<float4*>(dst)[i] =
+                                        make_float4(accf[4 * i], accf[4 * i + 1], accf[4 * i + 2], accf[4 * i + 3]);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 128; ++i)
+                                if (i < ncol) dst[i] = accf[i];
+                        }
+                    }
+                } else if constexpr (kMode == kModeUp) {
                     // h = bf16(silu(g) * u) for I-columns nt*128 + 64c + j, then the 1x128 FP8 quant of h
                     float amax = 0.0f;
 #pragma unroll
                     for (int j = 0; j < 64; ++j) {
-                        acc[j] = silu_mul(acc[j], acc[64 + j]);
-                        amax = fmaxf(amax, fabsf(acc[j]));
+                        accf[j] = silu_mul(accf[j], accf[64 + j]);
+                        amax = fmaxf(amax, fabsf(accf[j]));
                     }
                     amax_sh[c][r] = amax;
                     named_bar_sync(1, 256);
@@ -307,7 +362,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
 #pragma unroll
                                 for (int b = 0; b < 4; ++b) {
                                     const uint32_t code =
-                                        __nv_cvt_float_to_fp8(__fdiv_rn(acc[4 * i + b], sc), __NV_SATFINITE, __NV_E4M3);
+                                        __nv_cvt_float_to_fp8(__fdiv_rn(accf[4 * i + b], sc), __NV_SATFINITE, __NV_E4M3);
                                     word |= code << (8 * b);
                                 }
                             }
@@ -327,8 +382,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                         uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(grow) * out_ld + ti.nt * 256 + 128 * c) * 2);
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
-                            dst[i] = make_uint4(pack2(acc[8 * i], acc[8 * i + 1]), pack2(acc[8 * i + 2], acc[8 * i + 3]),
-                                                pack2(acc[8 * i + 4], acc[8 * i + 5]), pack2(acc[8 * i + 6], acc[8 * i + 7]));
+                            dst[i] = make_uint4(pack2(accf[8 * i], accf[8 * i + 1]), pack2(accf[8 * i + 2], accf[8 * i + 3]),
+                                                pack2(accf[8 * i + 4], accf[8 * i + 5]), pack2(accf[8 * i + 6], accf[8 * i + 7]));
                     }
                 }
             } else {
@@ -371,30 +426,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                                                     pack2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
                                                     pack2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
                                                     pack2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
-                        }
-                    }
-                } else {
-                    // router logits, float32, columns < n_valid_cols (a multiple of 8)
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint32_t v[32];
-                        tmem_ld32(base + 128 * c + 32 * ch, v);
-                        tmem_wait_ld();
-                        const int col0 = 128 * c + 32 * ch;
-                        if (valid) {
-                            float* dst = reinterpret_cast<float*>(out + (static_cast<size_t>(grow) * out_ld + col0) * 4);
-                            if ((p.n_valid_cols & 3) == 0) {        // rows 16-byte aligned: vector stores
-#pragma unroll
-                                for (int i = 0; i < 8; ++i)
-                                    if (col0 + 4 * i < p.n_valid_cols)
-                                        reinterpret_cast<float4*>(dst)[i] =
-                                            make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                                        __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-                            } else {
-#pragma unroll
-                                for (int i = 0; i < 32; ++i)
-                                    if (col0 + i < p.n_valid_cols) dst[i] = __uint_as_float(v[i]);
-                            }
                         }
                     }
                 }

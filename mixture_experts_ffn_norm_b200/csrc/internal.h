@@ -15,7 +15,7 @@ constexpr int kBN = 256;          // columns (weight rows) per GEMM tile
 constexpr int kStageBytesA = kBM * 128;
 constexpr int kStageBytesB = kBN * 128;
 constexpr int kStages = 4;
-constexpr int kGemmThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kGemmThreads = 384;  // warpgroup 0: warp 0 TMA, warp 1 MMA; warpgroups 1-2: epilogue
 constexpr int kMaxExperts = 256;
 constexpr int kRouteChunk = 2048;  // (token, slot) entries per block in the routing kernels
 
