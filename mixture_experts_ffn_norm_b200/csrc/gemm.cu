@@ -20,6 +20,8 @@
 //   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=32 bytes per instruction)
 //   warps 2-3   idle (they only hand their registers back)
 //   warps 4..11 epilogue: warp w reads TMEM lanes 32*(w%4).., column half (w-4)/4
+// The MMA thread and the epilogue poll their barriers (mbar_spin) rather than suspend in try_wait:
+// the TMEM double buffer makes their handshake the critical path, and a suspended waiter wakes late.
 // setmaxnreg moves registers from warpgroup 0 (56 each) to the two epilogue warpgroups (224 each):
 // 128*56 + 256*224 = 64512 = 384 * 168, the launch budget.  The FP8 promotion keeps 128 float32
 // accumulators per thread, loads 64 TMEM columns per wait, accumulates with packed fp32x2 FMAs and
@@ -206,13 +208,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                 decode_tile(t, ts_sh, rb_sh, rc_sh, p, kMode, ti);
                 for (int kb = 0; kb < ti.kb; ++kb) {
                     if (kPromote || kb == 0) {
-                        if (!mbar_wait(&tempty_bar[abuf], aphase ^ 1u, &abort_sh, p.status, 0x20)) {
+                        if (!mbar_spin(&tempty_bar[abuf], aphase ^ 1u, &abort_sh, p.status, 0x20)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                     }
-                    if (!mbar_wait(&full_bar[stage], phase, &abort_sh, p.status, 0x21)) {
+                    if (!mbar_spin(&full_bar[stage], phase, &abort_sh, p.status, 0x21)) {
                         ok = false;
                         break;
                     }
@@ -285,7 +287,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                         w0_n = __ldg(sc0 + kn);
                         w1_n = (kMode == kModeUp) ? __ldg(sc1 + kn) : 0.0f;
                     }
-                    if (!mbar_wait(&tfull_bar[abuf], aphase, &abort_sh, p.status, 0x30)) {
+                    if (!mbar_spin(&tfull_bar[abuf], aphase, &abort_sh, p.status, 0x30)) {
                         ok = false;
                         break;
                     }
@@ -388,7 +390,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                 }
             } else {
                 // bf16: the whole K accumulated in TMEM buffer abuf
-                if (!mbar_wait(&tfull_bar[abuf], aphase, &abort_sh, p.status, 0x31)) break;
+                if (!mbar_spin(&tfull_bar[abuf], aphase, &abort_sh, p.status, 0x31)) break;
                 tc_fence_after();
                 const uint32_t base = tl + static_cast<uint32_t>(abuf * kBN);
                 if constexpr (kMode == kModeUp) {
