@@ -58,6 +58,20 @@ bool encode_map_2d(CUtensorMap* map, const void* base, bool fp8, uint64_t inner,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_store_map_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
+                         uint32_t box_inner) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elem_bytes)};
+    const cuuint32_t box[2] = {box_inner, 32u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(map, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_layout(const moe_config_t& c, Layout& L) {
     if (c.num_tokens < 1 || c.dim < 256 || c.dim % 256 || c.inter_dim < 128 || c.inter_dim % 128) return false;
     if (c.n_experts < 1 || c.n_experts > kMaxExperts || (c.n_experts > 8 && c.n_experts % 8)) return false;
@@ -199,6 +213,8 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
         m.b1_s = m.b0_s;
         m.b0_r = m.b0_s;
         m.b1_r = m.b0_s;
+        m.o_r = m.a_s;
+        m.o_s = m.a_s;
         GemmParams p{};
         p.G = 1;
         p.single_rows = L.T;
@@ -236,6 +252,13 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
             ok = ok && encode_map_2d(&m.b0_s, w->sw1, fp8, L.d, L.Is) && encode_map_2d(&m.b1_s, w->sw3, fp8, L.d, L.Is);
         else
             m.b0_s = m.b0_r, m.b1_s = m.b1_r;
+        if (fp8) {
+            ok = ok && encode_store_map_2d(&m.o_r, ws + L.h, 1, L.I, L.R, 64);
+            if (L.Is > 0) ok = ok && encode_store_map_2d(&m.o_s, ws + L.h_sh, 1, L.Is, L.Tpad, 64);
+            else m.o_s = m.o_r;
+        } else {
+            m.o_r = m.a_r, m.o_s = m.a_r;
+        }
         if (!ok) return MOE_ERR_CUDA;
         GemmParams p{};
         p.G = G;
@@ -281,6 +304,13 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
             m.b1_s = m.b0_s;
         } else {
             m.a_s = m.a_r, m.b0_s = m.b0_r, m.b1_s = m.b0_r;
+        }
+        if (fp8) {
+            ok = ok && encode_store_map_2d(&m.o_r, ws + L.y, 2, L.d, L.R, 32);
+            if (L.Is > 0) ok = ok && encode_store_map_2d(&m.o_s, ws + L.y_sh, 2, L.d, L.T, 32);
+            else m.o_s = m.o_r;
+        } else {
+            m.o_r = m.a_r, m.o_s = m.a_r;
         }
         if (!ok) return MOE_ERR_CUDA;
         GemmParams p{};

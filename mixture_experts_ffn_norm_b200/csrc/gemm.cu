@@ -40,7 +40,8 @@ namespace moe {
 namespace {
 
 constexpr int kStageBytes = kStageBytesA + kStageBytesB;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+constexpr int kOutStageBytes = 2048;                       // per epilogue warp: 32 rows x 64 bytes
+constexpr int kSmemBytes = kStages * kStageBytes + 8 * kOutStageBytes + 1024;
 constexpr uint32_t kTmemCols = 512;
 
 struct Tile {
@@ -83,10 +84,28 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
            (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(b))) << 16);
 }
 
+// a / b given y = the correctly rounded 1/b: one product and one FMA-residual correction
+// (Markstein), which yields the correctly rounded quotient -- exact quotients, such as the
+// e4m3 rounding midpoints a group quantisation often lands on, come out exact.
+__device__ __forceinline__ float div_by_rcp(float a, float b, float y) {
+    const float q = a * y;
+    return fmaf(fmaf(-q, b, a), y, q);
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ float silu_mul(float g, float u) {
-    // silu(g) * u with the Linear outputs g, u in bf16 and the product rounded to bf16
+    // silu(g) * u with the Linear outputs g, u in bf16 and the product rounded to bf16; silu in
+    // float32: expf and a corrected division (1 + e >= 1, so the approximate reciprocal is safe)
     const float gb = bf16r(g), ub = bf16r(u);
-    return bf16r((gb / (1.0f + expf(-gb))) * ub);
+    const float d = 1.0f + expf(-gb);
+    // exp overflow (g below about -88): silu(g) rounds to zero; the correction step would form 0 * inf
+    const float sg = d < INFINITY ? div_by_rcp(gb, d, rcp_approx(d)) : 0.0f;
+    return bf16r(sg * ub);
 }
 
 template <bool kFp8, int kMode>
@@ -94,6 +113,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ CUtensorMap tm_a_s,
             const __grid_constant__ CUtensorMap tm_b0_r, const __grid_constant__ CUtensorMap tm_b1_r,
             const __grid_constant__ CUtensorMap tm_b0_s, const __grid_constant__ CUtensorMap tm_b1_s,
+            const __grid_constant__ CUtensorMap tm_o_r, const __grid_constant__ CUtensorMap tm_o_s,
             const GemmParams p) {
     extern __shared__ uint8_t dyn_smem[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
@@ -248,6 +268,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
         const int q = warp & 3;
         const int c = (warp - 4) >> 2;
         const int r = q * 32 + lane;
+        uint8_t* ostage = smem + kStages * kStageBytes + (warp - 4) * kOutStageBytes;
         const uint32_t tl = tmem + (static_cast<uint32_t>(q * 32) << 16);
         int abuf = 0;
         uint32_t aphase = 0;
@@ -355,37 +376,59 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                     amax = fmaxf(amax, amax_sh[c ^ 1][r]);
                     named_bar_sync(1, 256);
                     const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-                    if (valid) {
-                        uint32_t w[16];
+                    const float rsc = __frcp_rn(sc);
+                    // the row's 64 e4m3 codes -> this warp's staging rows -> one TMA store of 32 x 64 bytes
+                    uint32_t w[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            uint32_t word = 0;
-                            if (amax > 0.0f) {
+                    for (int i = 0; i < 16; ++i) {
+                        uint32_t word = 0;
+                        if (amax > 0.0f) {
 #pragma unroll
-                                for (int b = 0; b < 4; ++b) {
-                                    const uint32_t code =
-                                        __nv_cvt_float_to_fp8(__fdiv_rn(accf[4 * i + b], sc), __NV_SATFINITE, __NV_E4M3);
-                                    word |= code << (8 * b);
-                                }
+                            for (int b = 0; b < 4; ++b) {
+                                const uint32_t code =
+                                    __nv_cvt_float_to_fp8(div_by_rcp(accf[4 * i + b], sc, rsc), __NV_SATFINITE, __NV_E4M3);
+                                word |= code << (8 * b);
                             }
-                            w[i] = word;
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(grow) * out_ld + ti.nt * 128 + 64 * c);
+                        w[i] = word;
+                    }
+                    if (lane == 0) bulk_wait_read();
+                    __syncwarp();
+                    uint4* srow = reinterpret_cast<uint4*>(ostage + lane * 64);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-                        if (c == 0) {
-                            float* os = ti.shared ? p.outs_s : p.outs_r;
-                            const size_t os_ld = static_cast<size_t>(ti.shared ? p.outs_ld_s : p.outs_ld_r);
-                            os[static_cast<size_t>(ti.nt) * os_ld + grow] = sc;
-                        }
+                    for (int i = 0; i < 4; ++i) srow[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    fence_async_shared();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(ti.shared ? &tm_o_s : &tm_o_r, ostage, ti.nt * 128 + 64 * c, ti.a_row0 + q * 32);
+                        bulk_commit();
+                    }
+                    if (valid && c == 0) {
+                        float* os = ti.shared ? p.outs_s : p.outs_r;
+                        const size_t os_ld = static_cast<size_t>(ti.shared ? p.outs_ld_s : p.outs_ld_r);
+                        os[static_cast<size_t>(ti.nt) * os_ld + grow] = sc;
                     }
                 } else {
-                    if (valid) {
-                        uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(grow) * out_ld + ti.nt * 256 + 128 * c) * 2);
+                    // y rows (bf16): 4 chunks of 32 columns, each through this warp's staging rows and
+                    // one TMA store of 32 x 32 bf16
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            dst[i] = make_uint4(pack2(accf[8 * i], accf[8 * i + 1]), pack2(accf[8 * i + 2], accf[8 * i + 3]),
-                                                pack2(accf[8 * i + 4], accf[8 * i + 5]), pack2(accf[8 * i + 6], accf[8 * i + 7]));
+                    for (int ch = 0; ch < 4; ++ch) {
+                        if (lane == 0) bulk_wait_read();
+                        __syncwarp();
+                        uint4* srow = reinterpret_cast<uint4*>(ostage + lane * 64);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float* a8 = accf + ch * 32 + 8 * i;
+                            srow[i] = make_uint4(pack2(a8[0], a8[1]), pack2(a8[2], a8[3]), pack2(a8[4], a8[5]),
+                                                 pack2(a8[6], a8[7]));
+                        }
+                        fence_async_shared();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(ti.shared ? &tm_o_s : &tm_o_r, ostage, ti.nt * 256 + 128 * c + 32 * ch,
+                                         ti.a_row0 + q * 32);
+                            bulk_commit();
+                        }
                     }
                 }
             } else {
@@ -440,6 +483,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
         }
     }
 
+    if (warp >= 4 && lane == 0) bulk_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -453,7 +497,8 @@ cudaError_t launch_one(const TensorMaps& m, const GemmParams& p, int grid, cudaS
     cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kFp8, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemBytes);
     if (e != cudaSuccess) return e;
-    gemm_kernel<kFp8, kMode><<<grid, kGemmThreads, kSmemBytes, s>>>(m.a_r, m.a_s, m.b0_r, m.b1_r, m.b0_s, m.b1_s, p);
+    gemm_kernel<kFp8, kMode><<<grid, kGemmThreads, kSmemBytes, s>>>(m.a_r, m.a_s, m.b0_r, m.b1_r, m.b0_s, m.b1_s,
+                                                                     m.o_r, m.o_s, p);
     return cudaGetLastError();
 }
 

@@ -62,10 +62,14 @@ struct GemmParams {
 
 struct TensorMaps {
     CUtensorMap a_r, a_s, b0_r, b1_r, b0_s, b1_s;
+    CUtensorMap o_r, o_s;   // FP8 epilogue outputs (h or y rows), written by TMA stores
 };
 
 // tensor-map encoding (driver entry point fetched at run time; no libcuda link)
 bool encode_map_2d(CUtensorMap* map, const void* base, bool fp8, uint64_t inner, uint64_t rows);
+// unswizzled map for TMA stores of [32 rows x box_inner elements] boxes
+bool encode_store_map_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
+                         uint32_t box_inner);
 
 cudaError_t launch_norm(const Layout& L, const void* x, const void* residual, const float* g, float eps,
                         void* residual_out, uint8_t* ws, cudaStream_t s);
