@@ -179,6 +179,15 @@ moe_status_t moe_route_noalloc(const int32_t* idx, int32_t num_tokens, int32_t t
                                int32_t* counts, int32_t* offsets, int32_t* row_of, int32_t* row_token,
                                void* stream);
 
+/* Failure-detection self-test (the pages have no counterpart).  Enqueues one kernel whose only
+ * wait is on a barrier that is never signalled, using the same bounded wait as the pipeline
+ * kernels with a limit of `limit_cycles` SM clocks (1 .. 2^31).  The wait gives up, the kernel
+ * latches MOE_ERR_DEVICE_TIMEOUT into the status word at the start of `workspace` and returns
+ * normally; moe_get_status then reports MOE_ERR_DEVICE_TIMEOUT and the context stays usable.
+ * The next moe_forward on the workspace clears the status.  workspace_bytes >= 256. */
+moe_status_t moe_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int64_t limit_cycles,
+                                       void* stream);
+
 /* Number of kernel launches one moe_forward enqueues for this configuration. */
 int32_t moe_launches_per_forward(const moe_config_t* cfg);
 

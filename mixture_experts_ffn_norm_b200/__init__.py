@@ -20,7 +20,8 @@ MOE_W_BF16, MOE_W_FP8_E4M3_B128 = 0, 1
 MOE_ACT_FP8_1x128, MOE_ACT_BF16 = 0, 1
 
 EXPORTS = ("moe_workspace_bytes", "moe_forward", "moe_forward_traced", "moe_get_status", "moe_debug_routing",
-           "moe_debug_norm", "moe_route_noalloc", "moe_launches_per_forward", "moe_status_string")
+           "moe_debug_norm", "moe_route_noalloc", "moe_selftest_wait_timeout", "moe_launches_per_forward",
+           "moe_status_string")
 
 
 class MoeError(RuntimeError):
@@ -65,6 +66,8 @@ def lib() -> C.CDLL:
         L.moe_debug_norm.argtypes = [cfgp, vp, vp, vp, vp, vp]
         L.moe_route_noalloc.restype = C.c_int
         L.moe_route_noalloc.argtypes = [vp, C.c_int32, C.c_int32, C.c_int32, vp, vp, vp, vp, vp]
+        L.moe_selftest_wait_timeout.restype = C.c_int
+        L.moe_selftest_wait_timeout.argtypes = [vp, C.c_size_t, C.c_int64, vp]
         L.moe_launches_per_forward.restype = C.c_int32
         L.moe_launches_per_forward.argtypes = [cfgp]
         L.moe_status_string.restype = C.c_char_p
@@ -166,6 +169,12 @@ def moe_debug_norm(cfg: Config, workspace, xn=None, xq=None, xs=None, stream=Non
     rc = lib().moe_debug_norm(C.byref(cfg.c()), _ptr(workspace), _ptr(xn), _ptr(xq), _ptr(xs), _stream(stream))
     if rc != MOE_OK:
         raise MoeError(rc, "moe_debug_norm")
+
+
+def moe_selftest_wait_timeout(workspace, limit_cycles: int = 1 << 21, stream=None) -> int:
+    """Run the bounded-wait self-test on ``workspace`` (see include/moe.h); returns the call status."""
+    return int(lib().moe_selftest_wait_timeout(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                                limit_cycles, _stream(stream)))
 
 
 def route_rows(num_tokens: int, top_k: int, n_experts: int) -> int:

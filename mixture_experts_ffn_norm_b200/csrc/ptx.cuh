@@ -51,14 +51,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait until the phase with `parity` of the barrier has completed.  Returns false when the CTA
 // was told to abort or the wait ran out (then the abort flag is raised and the error latched).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status, uint32_t where) {
+                                          uint32_t* status, uint32_t where, long long limit = kWaitCycles) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(a, parity)) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             latch_error(status, kErrTimeout, where);
             return false;
