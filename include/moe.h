@@ -72,7 +72,7 @@ typedef enum {
 
 typedef struct {
     int32_t num_tokens;    /* T = B * S, >= 1 */
-    int32_t dim;           /* d, multiple of 256 */
+    int32_t dim;           /* d, multiple of 256, at most 8192 */
     int32_t inter_dim;     /* I (moe_inter_dim), multiple of 128 */
     int32_t n_experts;     /* E routed experts, 1..256, multiple of 8 or E <= 8 */
     int32_t top_k;         /* k, 1..E */

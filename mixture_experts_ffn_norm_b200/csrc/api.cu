@@ -73,7 +73,8 @@ bool encode_store_map_2d(CUtensorMap* map, const void* base, int elem_bytes, uin
 }
 
 bool make_layout(const moe_config_t& c, Layout& L) {
-    if (c.num_tokens < 1 || c.dim < 256 || c.dim % 256 || c.inter_dim < 128 || c.inter_dim % 128) return false;
+    if (c.num_tokens < 1 || c.dim < 256 || c.dim % 256 || c.dim > 8192 || c.inter_dim < 128 || c.inter_dim % 128)
+        return false;
     if (c.n_experts < 1 || c.n_experts > kMaxExperts || (c.n_experts > 8 && c.n_experts % 8)) return false;
     if (c.top_k < 1 || c.top_k > c.n_experts) return false;
     if (c.shared_inter < 0 || c.shared_inter % 128) return false;

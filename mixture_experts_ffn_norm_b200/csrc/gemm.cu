@@ -20,6 +20,7 @@
 //   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=32 bytes per instruction)
 //   warps 2-3   idle (they only hand their registers back)
 //   warps 4..11 epilogue: warp w reads TMEM lanes 32*(w%4).., column half (w-4)/4
+// Each promotion reads 64 TMEM columns per tcgen05.ld (two per K block per thread).
 // The MMA thread and the epilogue poll their barriers (mbar_spin) rather than suspend in try_wait:
 // the TMEM double buffer makes their handshake the critical path, and a suspended waiter wakes late.
 // setmaxnreg moves registers from warpgroup 0 (56 each) to the two epilogue warpgroups (224 each):
@@ -319,25 +320,29 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                     const uint32_t base = tl + static_cast<uint32_t>(abuf * kBN);
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
-                        // UP: hh 0 = g columns (64c..), hh 1 = u columns (128+64c..); DOWN: 128c + 64hh
+                        // UP: hh 0 = g columns (64c..), hh 1 = u columns (128+64c..); DOWN / logits: 128c + 64hh
                         const int col = (kMode == kModeUp) ? (hh ? 128 : 0) + 64 * c : 128 * c + 64 * hh;
-                        uint32_t v0[32], v1[32];
-                        tmem_ld32(base + col, v0);
-                        tmem_ld32(base + col + 32, v1);
+                        uint32_t v[64];
+                        tmem_ld64(base + col, v);
                         tmem_wait_ld();
+                        if (kMode == kModeDown && hh == 1) {
+                            // down GEMM: hand the buffer back before the last FMAs (measured faster there;
+                            // the up GEMM's longer tiles do better releasing after them)
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&tempty_bar[abuf]);
+                        }
                         const float2 fv = hh ? f1v : f0v;
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            acc[hh * 32 + j] = __ffma2_rn(make_float2(__uint_as_float(v0[2 * j]), __uint_as_float(v0[2 * j + 1])),
-                                                          fv, acc[hh * 32 + j]);
-                            acc[hh * 32 + 16 + j] = __ffma2_rn(
-                                make_float2(__uint_as_float(v1[2 * j]), __uint_as_float(v1[2 * j + 1])), fv,
-                                acc[hh * 32 + 16 + j]);
-                        }
+                        for (int j = 0; j < 32; ++j)
+                            acc[hh * 32 + j] =
+                                __ffma2_rn(make_float2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])), fv, acc[hh * 32 + j]);
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty_bar[abuf]);
+                    if (kMode != kModeDown) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty_bar[abuf]);
+                    }
                     abuf ^= 1;
                     if (abuf == 0) aphase ^= 1u;
                     sa = sa_n;
