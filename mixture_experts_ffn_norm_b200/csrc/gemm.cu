@@ -16,8 +16,9 @@
 // promoted.  bf16 operands simply accumulate the whole K in TMEM.
 //
 // Warp roles (384 threads = 3 warpgroups, one CTA per SM, persistent over a device-side tile table):
-//   warp 0      one thread issues the TMA loads of A (128 x 128 B) and B (256 x 128 B) per stage
-//   warp 1      one thread issues tcgen05.mma (M=128, N=256, K=32 bytes per instruction)
+//   warp 0      issues the TMA loads of A (128 x 128 B) and B (256 x 128 B) per stage (one elected lane)
+//   warp 1      issues tcgen05.mma (M=128, N=256, K=32 bytes per instruction): the whole warp runs the
+//               loop and waits, one elected lane issues
 //   warps 2-3   idle (they only hand their registers back)
 //   warps 4..11 epilogue: warp w reads TMEM lanes 32*(w%4).., column half (w-4)/4
 // Each promotion reads 64 TMEM columns per tcgen05.ld (two per K block per thread).
@@ -175,28 +176,33 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
       regs_dec<56>();
       if (warp == 0) {
         // ------------------------------------------------------------------ TMA producer
-        if (lane == 0) {
+        // whole warp in the loop (warp-uniform coordinates), the elected lane issues
+        const bool leader = elect_one();
+        if (leader) {
             prefetch_tensormap(&tm_a_r);
             prefetch_tensormap(&tm_a_s);
             prefetch_tensormap(&tm_b0_r);
             prefetch_tensormap(&tm_b1_r);
             prefetch_tensormap(&tm_b0_s);
             prefetch_tensormap(&tm_b1_s);
-            int stage = 0;
-            uint32_t phase = 0, pend = 0, pend_par = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                Tile ti;
-                decode_tile(t, ts_sh, rb_sh, rc_sh, p, kMode, ti);
-                const CUtensorMap* ma = ti.shared ? &tm_a_s : &tm_a_r;
-                const CUtensorMap* mb0 = ti.shared ? &tm_b0_s : &tm_b0_r;
-                const CUtensorMap* mb1 = ti.shared ? &tm_b1_s : &tm_b1_r;
-                const int b1_row = (kMode == kModeUp) ? ti.b_row0 : ti.b_row0 + 128;
-                for (int kb = 0; kb < ti.kb; ++kb) {
-                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, p.status, 0x10)) {
-                        ok = false;
-                        break;
-                    }
+        }
+        int stage = 0;
+        uint32_t phase = 0, pend = 0, pend_par = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            Tile ti;
+            decode_tile(t, ts_sh, rb_sh, rc_sh, p, kMode, ti);
+            const CUtensorMap* ma = ti.shared ? &tm_a_s : &tm_a_r;
+            const CUtensorMap* mb0 = ti.shared ? &tm_b0_s : &tm_b0_r;
+            const CUtensorMap* mb1 = ti.shared ? &tm_b1_s : &tm_b1_r;
+            const int b1_row = (kMode == kModeUp) ? ti.b_row0 : ti.b_row0 + 128;
+            for (int kb = 0; kb < ti.kb; ++kb) {
+                const bool got = mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_sh, p.status, 0x10);
+                if (!__all_sync(0xFFFFFFFFu, got)) {
+                    ok = false;
+                    break;
+                }
+                if (leader) {
                     uint8_t* sa = smem + stage * kStageBytes;
                     uint8_t* sb = sa + kStageBytesA;
                     mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
@@ -204,64 +210,75 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                     tma_load_2d(sa, ma, &full_bar[stage], kx, ti.a_row0);
                     tma_load_2d(sb, mb0, &full_bar[stage], kx, ti.b_row0);
                     tma_load_2d(sb + 128 * 128, mb1, &full_bar[stage], kx, b1_row);
-                    pend |= 1u << stage;
-                    pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                }
+                __syncwarp();
+                pend |= 1u << stage;
+                pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
-            if (!ok)
-                for (int s = 0; s < kStages; ++s)
-                    if ((pend >> s) & 1u) drain_wait(&full_bar[s], (pend_par >> s) & 1u);
         }
+        if (!ok && leader)
+            for (int s = 0; s < kStages; ++s)
+                if ((pend >> s) & 1u) drain_wait(&full_bar[s], (pend_par >> s) & 1u);
+        __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = instr_desc(kFp8, kBM, kBN);
-            constexpr bool kPromote = kFp8 || kMode == kModeLogits;
-            int stage = 0, abuf = 0;
-            uint32_t phase = 0, aphase = 0;
-            bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                Tile ti;
-                decode_tile(t, ts_sh, rb_sh, rc_sh, p, kMode, ti);
-                for (int kb = 0; kb < ti.kb; ++kb) {
-                    if (kPromote || kb == 0) {
-                        if (!mbar_spin(&tempty_bar[abuf], aphase ^ 1u, &abort_sh, p.status, 0x20)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                    }
-                    if (!mbar_spin(&full_bar[stage], phase, &abort_sh, p.status, 0x21)) {
+        // The whole warp runs the loop, so the descriptors are warp-uniform; the elected lane issues
+        // the MMAs and the commits (a commit tracks the MMAs of the thread that issues it).
+        constexpr uint32_t idesc = instr_desc(kFp8, kBM, kBN);
+        constexpr bool kPromote = kFp8 || kMode == kModeLogits;
+        const bool leader = elect_one();
+        int stage = 0, abuf = 0;
+        uint32_t phase = 0, aphase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            Tile ti;
+            decode_tile(t, ts_sh, rb_sh, rc_sh, p, kMode, ti);
+            for (int kb = 0; kb < ti.kb; ++kb) {
+                // the operands are normally resident long before the accumulator buffer is handed back,
+                // so everything but the TMEM-empty wait is done first: the MMAs follow that wait directly
+                if (!mbar_spin_warp(&full_bar[stage], phase, &abort_sh, p.status, 0x21)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+                const uint64_t ad = smem_desc_sw128(sa);
+                const uint64_t bd = smem_desc_sw128(sa + kStageBytesA);
+                const uint32_t dt = tmem + static_cast<uint32_t>(abuf * kBN);
+                const bool last = kPromote || kb == ti.kb - 1;
+                if (kPromote || kb == 0) {
+                    if (!mbar_spin_warp(&tempty_bar[abuf], aphase ^ 1u, &abort_sh, p.status, 0x20)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    const uint32_t sa = smem_u32(smem + stage * kStageBytes);
-                    const uint64_t ad = smem_desc_sw128(sa);
-                    const uint64_t bd = smem_desc_sw128(sa + kStageBytesA);
-                    const uint32_t dt = tmem + static_cast<uint32_t>(abuf * kBN);
+                }
+                tc_fence_after();
+                if (leader) {
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         umma<kFp8>(dt, ad + 2 * ks, bd + 2 * ks, idesc, kPromote ? (ks > 0) : (kb > 0 || ks > 0));
                     umma_commit(&empty_bar[stage]);
-                    if (kPromote || kb == ti.kb - 1) {
-                        umma_commit(&tfull_bar[abuf]);
-                        abuf ^= 1;
-                        if (abuf == 0) aphase ^= 1u;
-                    }
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    if (last) umma_commit(&tfull_bar[abuf]);
+                }
+                __syncwarp();
+                if (last) {
+                    abuf ^= 1;
+                    if (abuf == 0) aphase ^= 1u;
+                }
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
                 }
             }
+        }
+        if (leader) {
             umma_commit(&drain_bar);
             drain_wait(&drain_bar, 0);
         }
+        __syncwarp();
       }
     } else {
         regs_inc<224>();

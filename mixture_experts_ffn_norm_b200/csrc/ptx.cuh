@@ -98,6 +98,23 @@ __device__ __forceinline__ bool mbar_spin(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// mbar_spin run by every lane of a warp, with a warp-uniform result: the caller's control flow
+// stays convergent, so the operands it computes next are warp-uniform.
+__device__ __forceinline__ bool mbar_spin_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               uint32_t* status, uint32_t where) {
+    const bool r = mbar_spin(bar, parity, abort_flag, status, where);
+    return __all_sync(0xFFFFFFFFu, r);
+}
+
+// One lane of a fully active warp (the same lane on every call), chosen by elect.sync.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t e;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(e));
+    return e != 0;
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
