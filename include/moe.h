@@ -63,8 +63,10 @@ typedef enum {
 
 /* Precision of the activations fed to the expert GEMMs (the FP8 GEMM body is not on the
  * pages).  MOE_ACT_FP8_1x128: per token and per 128-column group, sc = amax/448,
- * q = e4m3(v/sc) -- applied to the normed input and to the SwiGLU hidden state h.
- * MOE_ACT_BF16: bf16 activations (the only mode for bf16 weights). */
+ * q = e4m3(v/sc) -- applied to the normed input and to the SwiGLU hidden state h; FP8 tensor-core
+ * GEMMs.  MOE_ACT_BF16: bf16 activations -- the only mode for bf16 weights; with FP8 weights, the
+ * plain reading of a block-scaled FP8 Linear: bf16 activations times the dequantised weights, each
+ * e4m3 weight tile widened to bf16 on chip and the block scales applied to the float32 partials. */
 typedef enum {
     MOE_ACT_FP8_1x128 = 0,
     MOE_ACT_BF16 = 1
@@ -80,7 +82,7 @@ typedef struct {
                               shared experts are one SwiGLU with concatenated hidden units);
                               multiple of 128; 0 = no shared expert */
     int32_t wtype;         /* moe_wtype_t, same for routed and shared weights */
-    int32_t amode;         /* moe_amode_t; FP8 weights need MOE_ACT_FP8_1x128 in this build */
+    int32_t amode;         /* moe_amode_t; bf16 weights need MOE_ACT_BF16 */
     float eps;             /* RMSNorm eps (1e-6 on the pages) */
 } moe_config_t;
 

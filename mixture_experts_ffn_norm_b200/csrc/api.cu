@@ -58,6 +58,18 @@ bool encode_map_2d(CUtensorMap* map, const void* base, bool fp8, uint64_t inner,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_raw_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner};
+    const cuuint32_t box[2] = {64u, 128u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_store_map_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
                          uint32_t box_inner) {
     EncodeTiledFn enc = get_encode();
@@ -89,7 +101,7 @@ bool make_layout(const moe_config_t& c, Layout& L) {
     L.k = c.top_k;
     L.Is = c.shared_inter;
     L.fp8 = c.wtype == MOE_W_FP8_E4M3_B128;
-    L.act8 = L.fp8;
+    L.act8 = L.fp8 && c.amode == MOE_ACT_FP8_1x128;
     L.Tpad = static_cast<int>(align_up(L.T, kBM));
     L.R = static_cast<int>(align_up(static_cast<size_t>(L.T) * L.k + static_cast<size_t>(L.E) * (kBM - 1), kBM));
     L.KBd = L.d / 128;
@@ -141,7 +153,6 @@ namespace {
 moe_status_t check_config(const moe_config_t* cfg, Layout& L) {
     if (!cfg || !make_layout(*cfg, L)) return MOE_ERR_INVALID_ARG;
     if (cfg->wtype == MOE_W_BF16 && cfg->amode != MOE_ACT_BF16) return MOE_ERR_INVALID_ARG;
-    if (cfg->wtype == MOE_W_FP8_E4M3_B128 && cfg->amode != MOE_ACT_FP8_1x128) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
 
@@ -196,6 +207,8 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const int sms = num_sms();
     const bool fp8 = L.fp8;
+    const bool act8 = L.act8;           // FP8 activations into the expert GEMMs
+    const bool a16 = fp8 && !act8;      // FP8 weights widened to bf16 next to bf16 activations
 
     MOE_TRY(cudaMemsetAsync(ws + L.status, 0, kStatusWords * 4, s));
     MOE_TRY(cudaMemsetAsync(ws + L.row_token, 0xFF, static_cast<size_t>(L.R) * 4, s));
@@ -226,7 +239,7 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
         p.n_valid_cols = L.E;
         p.status = reinterpret_cast<uint32_t*>(ws + L.status);
         const int tiles = (L.T + kBM - 1) / kBM;
-        MOE_TRY(launch_gemm(kModeLogits, false, m, p, std::min(tiles, sms), s));
+        MOE_TRY(launch_gemm(kModeLogits, false, false, m, p, std::min(tiles, sms), s));
     }
     MOE_TRY(mark(2));
     // 3. top-k, re-decided in float64 near the boundary
@@ -245,15 +258,18 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
     // 5. grouped GEMM up: h = silu(a W1^T) * (a W3^T)
     {
         TensorMaps m;
-        bool ok = encode_map_2d(&m.a_r, ws + L.a_perm, fp8, L.d, L.R) &&
-                  encode_map_2d(&m.a_s, ws + (fp8 ? L.xq : L.xn), fp8, L.d, L.T) &&
-                  encode_map_2d(&m.b0_r, w->w1, fp8, L.d, static_cast<uint64_t>(L.E) * L.I) &&
-                  encode_map_2d(&m.b1_r, w->w3, fp8, L.d, static_cast<uint64_t>(L.E) * L.I);
+        auto bmap = [&](CUtensorMap* mp, const void* base, uint64_t inner, uint64_t rows) {
+            return a16 ? encode_raw_map_2d(mp, base, inner, rows) : encode_map_2d(mp, base, fp8, inner, rows);
+        };
+        bool ok = encode_map_2d(&m.a_r, ws + L.a_perm, act8, L.d, L.R) &&
+                  encode_map_2d(&m.a_s, ws + (act8 ? L.xq : L.xn), act8, L.d, L.T) &&
+                  bmap(&m.b0_r, w->w1, L.d, static_cast<uint64_t>(L.E) * L.I) &&
+                  bmap(&m.b1_r, w->w3, L.d, static_cast<uint64_t>(L.E) * L.I);
         if (L.Is > 0)
-            ok = ok && encode_map_2d(&m.b0_s, w->sw1, fp8, L.d, L.Is) && encode_map_2d(&m.b1_s, w->sw3, fp8, L.d, L.Is);
+            ok = ok && bmap(&m.b0_s, w->sw1, L.d, L.Is) && bmap(&m.b1_s, w->sw3, L.d, L.Is);
         else
             m.b0_s = m.b0_r, m.b1_s = m.b1_r;
-        if (fp8) {
+        if (act8) {
             ok = ok && encode_store_map_2d(&m.o_r, ws + L.h, 1, L.I, L.R, 64);
             if (L.Is > 0) ok = ok && encode_store_map_2d(&m.o_s, ws + L.h_sh, 1, L.Is, L.Tpad, 64);
             else m.o_s = m.o_r;
@@ -269,7 +285,7 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
         p.row_count = reinterpret_cast<const int*>(ws + L.row_count);
         p.n_tiles_r = ntu_r;
         p.n_tiles_s = ntu_s;
-        p.kb_r = p.kb_s = fp8 ? L.d / 128 : L.d / 64;
+        p.kb_r = p.kb_s = act8 ? L.d / 128 : L.d / 64;
         p.b_rows_per_expert = L.I;
         p.as_r = reinterpret_cast<const float*>(ws + L.as_perm);
         p.as_s = reinterpret_cast<const float*>(ws + L.xs);
@@ -290,18 +306,21 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
         p.outs_ld_r = L.R;
         p.outs_ld_s = L.Tpad;
         p.status = reinterpret_cast<uint32_t*>(ws + L.status);
-        MOE_TRY(launch_gemm(kModeUp, fp8, m, p, std::min(max_tiles_up, sms), s));
+        MOE_TRY(launch_gemm(kModeUp, fp8, a16, m, p, std::min(max_tiles_up, sms), s));
     }
     MOE_TRY(mark(5));
     // 6. grouped GEMM down: y = h W2^T
     {
         TensorMaps m;
-        bool ok = encode_map_2d(&m.a_r, ws + L.h, fp8, L.I, L.R) &&
-                  encode_map_2d(&m.b0_r, w->w2, fp8, L.I, static_cast<uint64_t>(L.E) * L.d);
+        auto bmap = [&](CUtensorMap* mp, const void* base, uint64_t inner, uint64_t rows) {
+            return a16 ? encode_raw_map_2d(mp, base, inner, rows) : encode_map_2d(mp, base, fp8, inner, rows);
+        };
+        bool ok = encode_map_2d(&m.a_r, ws + L.h, act8, L.I, L.R) &&
+                  bmap(&m.b0_r, w->w2, L.I, static_cast<uint64_t>(L.E) * L.d);
         m.b1_r = m.b0_r;
         if (L.Is > 0) {
-            ok = ok && encode_map_2d(&m.a_s, ws + L.h_sh, fp8, L.Is, L.Tpad) &&
-                 encode_map_2d(&m.b0_s, w->sw2, fp8, L.Is, L.d);
+            ok = ok && encode_map_2d(&m.a_s, ws + L.h_sh, act8, L.Is, L.Tpad) &&
+                 bmap(&m.b0_s, w->sw2, L.Is, L.d);
             m.b1_s = m.b0_s;
         } else {
             m.a_s = m.a_r, m.b0_s = m.b0_r, m.b1_s = m.b0_r;
@@ -321,8 +340,8 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
         p.row_base = reinterpret_cast<const int*>(ws + L.row_base);
         p.row_count = reinterpret_cast<const int*>(ws + L.row_count);
         p.n_tiles_r = p.n_tiles_s = ntd;
-        p.kb_r = fp8 ? L.I / 128 : L.I / 64;
-        p.kb_s = fp8 ? L.Is / 128 : L.Is / 64;
+        p.kb_r = act8 ? L.I / 128 : L.I / 64;
+        p.kb_s = act8 ? L.Is / 128 : L.Is / 64;
         p.b_rows_per_expert = L.d;
         p.as_r = reinterpret_cast<const float*>(ws + L.hs);
         p.as_s = reinterpret_cast<const float*>(ws + L.hs_sh);
@@ -337,7 +356,7 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
         p.out_s = ws + L.y_sh;
         p.out_ld_r = p.out_ld_s = L.d;
         p.status = reinterpret_cast<uint32_t*>(ws + L.status);
-        MOE_TRY(launch_gemm(kModeDown, fp8, m, p, std::min(max_tiles_down, sms), s));
+        MOE_TRY(launch_gemm(kModeDown, fp8, a16, m, p, std::min(max_tiles_down, sms), s));
     }
     MOE_TRY(mark(6));
     // 7. weighted combine + shared add -> out

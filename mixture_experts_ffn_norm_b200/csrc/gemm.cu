@@ -42,8 +42,14 @@ namespace moe {
 namespace {
 
 constexpr int kStageBytes = kStageBytesA + kStageBytesB;
+// bf16-activation mode for FP8 weights: the weight tile of a 64-wide K stage arrives as e4m3 bytes
+// (256 rows x 64 B) next to the stage and is widened to bf16 in the stage's B area
+constexpr int kRawBytes = 256 * 64;
+constexpr int kStagesA16 = 3;
+constexpr int kStageBytesA16 = kStageBytes + kRawBytes;
 constexpr int kOutStageBytes = 2048;                       // per epilogue warp: 32 rows x 64 bytes
 constexpr int kSmemBytes = kStages * kStageBytes + 8 * kOutStageBytes + 1024;
+constexpr int kSmemBytesA16 = kStagesA16 * kStageBytesA16 + 8 * kOutStageBytes + 1024;
 constexpr uint32_t kTmemCols = 512;
 
 struct Tile {
@@ -110,7 +116,18 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
     return bf16r(sg * ub);
 }
 
-template <bool kFp8, int kMode>
+// two e4m3 codes (low byte first) -> two bf16 (low half first); exact: every e4m3 value is a bf16 value
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two) {
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+    return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// kFp8: the weights are e4m3 with 128x128 block scales.  kA16 (with kFp8): the activations stay bf16
+// and each weight tile is widened to bf16 in shared memory by warps 2-3 before bf16 MMAs; otherwise
+// FP8 weights meet 1x128-quantised FP8 activations in FP8 MMAs.
+template <bool kFp8, int kMode, bool kA16>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ CUtensorMap tm_a_s,
             const __grid_constant__ CUtensorMap tm_b0_r, const __grid_constant__ CUtensorMap tm_b1_r,
@@ -121,6 +138,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(8) uint64_t full_bar[kStages];
     __shared__ __align__(8) uint64_t empty_bar[kStages];
+    __shared__ __align__(8) uint64_t conv_bar[kStages];    // kA16: the stage's weight tile is widened
     __shared__ __align__(8) uint64_t tfull_bar[2];
     __shared__ __align__(8) uint64_t tempty_bar[2];
     __shared__ __align__(8) uint64_t drain_bar;
@@ -132,6 +150,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
     __shared__ float amax_sh[2][kBM];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr bool kAct8 = kFp8 && !kA16;               // FP8 activations, FP8 MMAs
+    constexpr int NS = kA16 ? kStagesA16 : kStages;     // pipeline stages
+    constexpr int SB = kA16 ? kStageBytesA16 : kStageBytes;
+    constexpr int KX = kAct8 ? 128 : 64;                // K elements per stage
+    static_assert(!kA16 || kFp8, "the bf16-activation mode is for FP8 weights");
 
     if (p.single_rows > 0) {
         if (threadIdx.x == 0) {
@@ -150,9 +173,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
         }
     }
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
+            mbar_init(&conv_bar[s], 64);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull_bar[b], 1);
@@ -203,33 +227,35 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                     break;
                 }
                 if (leader) {
-                    uint8_t* sa = smem + stage * kStageBytes;
-                    uint8_t* sb = sa + kStageBytesA;
-                    mbar_arrive_expect_tx(&full_bar[stage], kStageBytes);
-                    const int kx = kb * (kFp8 ? 128 : 64);
+                    uint8_t* sa = smem + stage * SB;
+                    uint8_t* sb = sa + (kA16 ? kStageBytes : kStageBytesA);   // kA16: the raw e4m3 area
+                    mbar_arrive_expect_tx(&full_bar[stage], kA16 ? kStageBytesA + kRawBytes : kStageBytes);
+                    const int kx = kb * KX;
                     tma_load_2d(sa, ma, &full_bar[stage], kx, ti.a_row0);
                     tma_load_2d(sb, mb0, &full_bar[stage], kx, ti.b_row0);
-                    tma_load_2d(sb + 128 * 128, mb1, &full_bar[stage], kx, b1_row);
+                    tma_load_2d(sb + (kA16 ? kRawBytes / 2 : 128 * 128), mb1, &full_bar[stage], kx, b1_row);
                 }
                 __syncwarp();
                 pend |= 1u << stage;
                 pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
-                if (++stage == kStages) {
+                if (++stage == NS) {
                     stage = 0;
                     phase ^= 1u;
                 }
             }
         }
         if (!ok && leader)
-            for (int s = 0; s < kStages; ++s)
+            for (int s = 0; s < NS; ++s)
                 if ((pend >> s) & 1u) drain_wait(&full_bar[s], (pend_par >> s) & 1u);
         __syncwarp();
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
         // The whole warp runs the loop, so the descriptors are warp-uniform; the elected lane issues
         // the MMAs and the commits (a commit tracks the MMAs of the thread that issues it).
-        constexpr uint32_t idesc = instr_desc(kFp8, kBM, kBN);
+        constexpr uint32_t idesc = instr_desc(kAct8, kBM, kBN);
         constexpr bool kPromote = kFp8 || kMode == kModeLogits;
+        // stages per promoted K block: FP8 weights carry one scale per 128 K, a bf16 stage is 64 wide
+        constexpr int kPer = kA16 ? 2 : 1;
         const bool leader = elect_one();
         int stage = 0, abuf = 0;
         uint32_t phase = 0, aphase = 0;
@@ -240,16 +266,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
             for (int kb = 0; kb < ti.kb; ++kb) {
                 // the operands are normally resident long before the accumulator buffer is handed back,
                 // so everything but the TMEM-empty wait is done first: the MMAs follow that wait directly
-                if (!mbar_spin_warp(&full_bar[stage], phase, &abort_sh, p.status, 0x21)) {
+                if (!mbar_spin_warp(kA16 ? &conv_bar[stage] : &full_bar[stage], phase, &abort_sh, p.status, 0x21)) {
                     ok = false;
                     break;
                 }
-                const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+                const uint32_t sa = smem_u32(smem + stage * SB);
                 const uint64_t ad = smem_desc_sw128(sa);
                 const uint64_t bd = smem_desc_sw128(sa + kStageBytesA);
                 const uint32_t dt = tmem + static_cast<uint32_t>(abuf * kBN);
-                const bool last = kPromote || kb == ti.kb - 1;
-                if (kPromote || kb == 0) {
+                const bool first = kPromote ? (kb % kPer == 0) : kb == 0;   // first stage into this buffer
+                const bool last = kPromote ? (kb % kPer == kPer - 1) : kb == ti.kb - 1;
+                if (first) {
                     if (!mbar_spin_warp(&tempty_bar[abuf], aphase ^ 1u, &abort_sh, p.status, 0x20)) {
                         ok = false;
                         break;
@@ -259,7 +286,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                 if (leader) {
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        umma<kFp8>(dt, ad + 2 * ks, bd + 2 * ks, idesc, kPromote ? (ks > 0) : (kb > 0 || ks > 0));
+                        umma<kAct8>(dt, ad + 2 * ks, bd + 2 * ks, idesc, !first || ks > 0);
                     umma_commit(&empty_bar[stage]);
                     if (last) umma_commit(&tfull_bar[abuf]);
                 }
@@ -268,7 +295,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                     abuf ^= 1;
                     if (abuf == 0) aphase ^= 1u;
                 }
-                if (++stage == kStages) {
+                if (++stage == NS) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -279,6 +306,46 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
             drain_wait(&drain_bar, 0);
         }
         __syncwarp();
+      } else if constexpr (kA16) {
+        // ------------------------------------------------------------------ weight widening (kA16)
+        // warps 2-3: the stage's e4m3 weight tile (256 rows x 64 B, as loaded) -> bf16 rows of 128 B in
+        // the 128-byte-swizzled K-major layout the MMA reads (16-byte unit u of row n at unit u ^ (n % 8))
+        const int ct = threadIdx.x - 64;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            Tile ti;
+            decode_tile(t, ts_sh, rb_sh, rc_sh, p, kMode, ti);
+            for (int kb = 0; kb < ti.kb; ++kb) {
+                const bool got = mbar_wait(&full_bar[stage], phase, &abort_sh, p.status, 0x40);
+                if (!__all_sync(0xFFFFFFFFu, got)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* raw = smem + stage * SB + kStageBytes;
+                uint8_t* bb = smem + stage * SB + kStageBytesA;
+#pragma unroll 2
+                for (int i = 0; i < kRawBytes / 16 / 64; ++i) {
+                    const int u = i * 64 + ct;          // 16-byte unit of the raw tile: row u / 4, quarter u % 4
+                    const int n = u >> 2, qd = u & 3;
+                    const uint4 v = *reinterpret_cast<const uint4*>(raw + n * 64 + qd * 16);
+                    const uint4 lo = make_uint4(e4m3x2_to_bf16x2(v.x), e4m3x2_to_bf16x2(v.x >> 16),
+                                                e4m3x2_to_bf16x2(v.y), e4m3x2_to_bf16x2(v.y >> 16));
+                    const uint4 hi = make_uint4(e4m3x2_to_bf16x2(v.z), e4m3x2_to_bf16x2(v.z >> 16),
+                                                e4m3x2_to_bf16x2(v.w), e4m3x2_to_bf16x2(v.w >> 16));
+                    uint8_t* row = bb + n * 128;
+                    *reinterpret_cast<uint4*>(row + (((2 * qd) ^ (n & 7)) << 4)) = lo;
+                    *reinterpret_cast<uint4*>(row + (((2 * qd + 1) ^ (n & 7)) << 4)) = hi;
+                }
+                fence_async_shared();   // the tensor core reads these bytes through the async proxy
+                mbar_arrive(&conv_bar[stage]);
+                if (++stage == NS) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
       }
     } else {
         regs_inc<224>();
@@ -286,7 +353,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
         const int q = warp & 3;
         const int c = (warp - 4) >> 2;
         const int r = q * 32 + lane;
-        uint8_t* ostage = smem + kStages * kStageBytes + (warp - 4) * kOutStageBytes;
+        uint8_t* ostage = smem + NS * SB + (warp - 4) * kOutStageBytes;
         const uint32_t tl = tmem + (static_cast<uint32_t>(q * 32) << 16);
         int abuf = 0;
         uint32_t aphase = 0;
@@ -298,8 +365,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
             uint8_t* out = static_cast<uint8_t*>(ti.shared ? p.out_s : p.out_r);
             const size_t out_ld = static_cast<size_t>(ti.shared ? p.out_ld_s : p.out_ld_r);
             if constexpr (kFp8 || kMode == kModeLogits) {
-                // promotion: every K stage arrives in its own TMEM buffer and is added into float32
-                // registers (FP8: scaled by s_act[row, kb] * s_w[blk, kb]; logits: scale 1)
+                // promotion: every 128-wide K block arrives in its own TMEM buffer and is added into float32
+                // registers (FP8 activations: scaled by s_act[row, kb] * s_w[blk, kb]; bf16 activations
+                // with FP8 weights: by s_w[blk, kb]; logits: scale 1, one 64-wide stage per block)
                 float2 acc[64];
 #pragma unroll
                 for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.0f, 0.0f);
@@ -313,16 +381,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                 // scales of K block 0; each iteration fetches the next block's before it waits
                 float sa = 1.0f, w0 = 1.0f, w1 = 1.0f;
                 if constexpr (kScaled) {
-                    sa = as[grow];
+                    if constexpr (kAct8) sa = as[grow];
                     w0 = __ldg(sc0);
                     w1 = (kMode == kModeUp) ? __ldg(sc1) : 0.0f;
                 }
+                const int npb = kA16 ? ti.kb / 2 : ti.kb;   // promoted K blocks
                 bool ok = true;
-                for (int kb = 0; kb < ti.kb; ++kb) {
-                    const int kn = kb + 1 < ti.kb ? kb + 1 : kb;
+                for (int kb = 0; kb < npb; ++kb) {
+                    const int kn = kb + 1 < npb ? kb + 1 : kb;
                     float sa_n = 1.0f, w0_n = 1.0f, w1_n = 1.0f;
                     if constexpr (kScaled) {
-                        sa_n = as[static_cast<size_t>(kn) * as_ld + grow];
+                        if constexpr (kAct8) sa_n = as[static_cast<size_t>(kn) * as_ld + grow];
                         w0_n = __ldg(sc0 + kn);
                         w1_n = (kMode == kModeUp) ? __ldg(sc1 + kn) : 0.0f;
                     }
@@ -383,6 +452,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
 #pragma unroll
                             for (int i = 0; i < 128; ++i)
                                 if (i < ncol) dst[i] = accf[i];
+                        }
+                    }
+                } else if constexpr (kMode == kModeUp && kA16) {
+                    // h = bf16(silu(g) * u) for I-columns nt*128 + 64c + j, stored as bf16 (no quant)
+                    if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(
+                            out + (static_cast<size_t>(grow) * out_ld + ti.nt * 128 + 64 * c) * 2);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            float h[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) h[e] = silu_mul(accf[8 * i + e], accf[64 + 8 * i + e]);
+                            dst[i] = make_uint4(pack2(h[0], h[1]), pack2(h[2], h[3]), pack2(h[4], h[5]), pack2(h[6], h[7]));
                         }
                     }
                 } else if constexpr (kMode == kModeUp) {
@@ -514,19 +596,26 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
     }
 }
 
-template <bool kFp8, int kMode>
+template <bool kFp8, int kMode, bool kA16 = false>
 cudaError_t launch_one(const TensorMaps& m, const GemmParams& p, int grid, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kFp8, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
+    constexpr int smem = kA16 ? kSmemBytesA16 : kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kFp8, kMode, kA16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
     if (e != cudaSuccess) return e;
-    gemm_kernel<kFp8, kMode><<<grid, kGemmThreads, kSmemBytes, s>>>(m.a_r, m.a_s, m.b0_r, m.b1_r, m.b0_s, m.b1_s,
-                                                                     m.o_r, m.o_s, p);
+    gemm_kernel<kFp8, kMode, kA16><<<grid, kGemmThreads, smem, s>>>(m.a_r, m.a_s, m.b0_r, m.b1_r, m.b0_s, m.b1_s,
+                                                                    m.o_r, m.o_s, p);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_gemm(int mode, bool fp8, const TensorMaps& maps, const GemmParams& p, int grid, cudaStream_t s) {
+cudaError_t launch_gemm(int mode, bool fp8, bool a16, const TensorMaps& maps, const GemmParams& p, int grid,
+                        cudaStream_t s) {
+    if (fp8 && a16) {
+        if (mode == kModeUp) return launch_one<true, kModeUp, true>(maps, p, grid, s);
+        if (mode == kModeDown) return launch_one<true, kModeDown, true>(maps, p, grid, s);
+        return cudaErrorInvalidValue;
+    }
     if (fp8) {
         if (mode == kModeUp) return launch_one<true, kModeUp>(maps, p, grid, s);
         if (mode == kModeDown) return launch_one<true, kModeDown>(maps, p, grid, s);

@@ -67,13 +67,17 @@ struct TensorMaps {
 
 // tensor-map encoding (driver entry point fetched at run time; no libcuda link)
 bool encode_map_2d(CUtensorMap* map, const void* base, bool fp8, uint64_t inner, uint64_t rows);
+// unswizzled map over a row-major [rows, inner] byte tensor loading [128 rows x 64 bytes] boxes
+bool encode_raw_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows);
 // unswizzled map for TMA stores of [32 rows x box_inner elements] boxes
 bool encode_store_map_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
                          uint32_t box_inner);
 
 cudaError_t launch_norm(const Layout& L, const void* x, const void* residual, const float* g, float eps,
                         void* residual_out, uint8_t* ws, cudaStream_t s);
-cudaError_t launch_gemm(int mode, bool fp8, const TensorMaps& maps, const GemmParams& p, int grid,
+// fp8: e4m3 weights with block scales; a16 (with fp8): bf16 activations, the weights widened in
+// shared memory (the B maps then load raw 64-byte x 128-row e4m3 boxes, see encode_raw_map_2d)
+cudaError_t launch_gemm(int mode, bool fp8, bool a16, const TensorMaps& maps, const GemmParams& p, int grid,
                         cudaStream_t s);
 cudaError_t launch_topk(const Layout& L, const void* gate_w, const float* gate_bias, uint8_t* ws, cudaStream_t s);
 cudaError_t launch_route(const Layout& L, int ntu_r, int ntu_s, int ntd_r, int ntd_s, uint8_t* ws,

@@ -73,9 +73,9 @@ class GpuRun:
         tie = torch.empty(T, dtype=torch.uint8, device=dev)
         moe.moe_debug_routing(self.cfg, self.layer.workspace, idx, w, cnt, tie)
         xn = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
-        fp8 = self.cfg.wtype == moe.MOE_W_FP8_E4M3_B128
-        xq = torch.empty(T, d, dtype=torch.uint8, device=dev) if fp8 else None
-        xs = torch.empty(d // 128, T, dtype=torch.float32, device=dev) if fp8 else None
+        act8 = self.cfg.wtype == moe.MOE_W_FP8_E4M3_B128 and self.cfg.amode == moe.MOE_ACT_FP8_1x128
+        xq = torch.empty(T, d, dtype=torch.uint8, device=dev) if act8 else None
+        xs = torch.empty(d // 128, T, dtype=torch.float32, device=dev) if act8 else None
         moe.moe_debug_norm(self.cfg, self.layer.workspace, xn, xq, xs)
         torch.cuda.synchronize()
         self.out = bits_np(out)

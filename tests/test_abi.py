@@ -1,6 +1,7 @@
 """The C ABI without a GPU: the library loads, exports every entry point include/moe.h declares,
 sizes workspaces, and rejects bad arguments synchronously (before any CUDA call)."""
 import ctypes as C
+import dataclasses
 import os
 import re
 
@@ -40,6 +41,9 @@ def test_workspace_sizes_and_invalid_configs():
         assert moe.launches_per_forward(cfg) == 10
     c4 = moe.Config.from_shape(synthetic.CONFIGS["C4"])
     assert moe.workspace_bytes(c4) < 8 * 2 ** 30
+    # bf16 activations with FP8 weights: the permuted rows and h are 2 bytes wide, no activation scales
+    c4_a16 = dataclasses.replace(c4, amode=moe.MOE_ACT_BF16)
+    assert moe.workspace_bytes(c4) < moe.workspace_bytes(c4_a16) < 2 * moe.workspace_bytes(c4)
     bad = [dict(dim=200), dict(inter_dim=100), dict(top_k=0), dict(top_k=300), dict(n_experts=300),
            dict(n_experts=12), dict(num_tokens=0), dict(shared_inter=64), dict(wtype=7)]
     for b in bad:
@@ -66,6 +70,11 @@ def test_forward_rejects_bad_arguments_without_touching_the_device():
     assert L.moe_forward(*args(out=fake)) == moe.MOE_ERR_INVALID_ARG            # out aliases x
     bad = moe.Config(64, 256, 128, 8, 9, 128, moe.MOE_W_BF16, moe.MOE_ACT_BF16).c()
     assert L.moe_forward(*args(cfg=bad)) == moe.MOE_ERR_INVALID_ARG
-    fp8_a16 = moe.Config(64, 256, 128, 8, 2, 128, moe.MOE_W_FP8_E4M3_B128, moe.MOE_ACT_BF16).c()
-    assert L.moe_forward(*args(cfg=fp8_a16)) == moe.MOE_ERR_UNSUPPORTED
+    # FP8 weights need their block scales, in either activation mode
+    for amode in (moe.MOE_ACT_FP8_1x128, moe.MOE_ACT_BF16):
+        fp8 = moe.Config(64, 256, 128, 8, 2, 128, moe.MOE_W_FP8_E4M3_B128, amode).c()
+        assert L.moe_forward(*args(cfg=fp8, wsb=L.moe_workspace_bytes(C.byref(fp8)))) == moe.MOE_ERR_INVALID_ARG
+    # bf16 weights with FP8 activations is not a mode
+    bf16_a8 = moe.Config(64, 256, 128, 8, 2, 128, moe.MOE_W_BF16, moe.MOE_ACT_FP8_1x128).c()
+    assert L.moe_forward(*args(cfg=bf16_a8)) == moe.MOE_ERR_INVALID_ARG
     assert moe.status_string(moe.MOE_ERR_WORKSPACE) == "workspace missing or too small"
