@@ -89,11 +89,11 @@ def make_inputs(shape, device):
 # ------------------------------------------------------------------------------------------------
 # algorithmic work
 # ------------------------------------------------------------------------------------------------
-def work(shape, counts):
+def work(shape, counts, act8=True):
     """FLOPs and bytes of one step and of the grouped GEMM up (the dominant kernel)."""
     T, d, I, E, k, Is = shape.T, shape.d, shape.I, shape.E, shape.k, shape.Is
     wb = 1 if shape.wtype == "fp8" else 2
-    ab = wb
+    ab = 1 if (wb == 1 and act8) else 2
     touched = int((np.asarray(counts) > 0).sum())
     scl = lambda r, c: (r // 128) * (c // 128) * 4 if wb == 1 else 0
     expert_bytes = 3 * d * I * wb + 2 * scl(I, d) + scl(d, I)
@@ -157,10 +157,10 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------------
 # CPU oracle timing
 # ------------------------------------------------------------------------------------------------
-def oracle_throughput(shape, inputs, budget_s=20.0, max_tokens=1024, seed=0):
+def oracle_throughput(shape, inputs, budget_s=20.0, max_tokens=1024, seed=0, act8=True):
     """Tokens/s of the oracle on a bounded seeded sample of the workload's tokens (all host cores)."""
     import oracle
-    o = oracle.Oracle(shape, inputs)
+    o = oracle.Oracle(shape, inputs, act_fp8=act8 and shape.wtype == "fp8")
     cores = oracle.default_threads()
     rng = np.random.default_rng(seed)
     n0 = min(shape.T, cores)
@@ -183,7 +183,7 @@ def run_reference(args, shape, rank):
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inputs = make_inputs(shape, dev)
     import oracle
-    o = oracle.Oracle(shape, inputs)
+    o = oracle.Oracle(shape, inputs, act_fp8=args.act == "fp8" and shape.wtype == "fp8")
     cores = oracle.default_threads()
     n = min(shape.T, max(1, cores))
     rng = np.random.default_rng(1)
@@ -197,19 +197,20 @@ def run_reference(args, shape, rank):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_block(shape),
+            "config": config_block(shape, args.act == "fp8"),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": f"{n} seeded tokens of {shape.T} per step, full layer per token"},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def config_block(shape):
+def config_block(shape, act8=True):
     desc = synthetic.DESCRIPTIONS.get(shape.name, "reduced case of " + shape.name.split("-")[0] + " (profiling only)")
     return {"workload": f"{shape.name}: {desc}", "tokens": shape.T, "dim": shape.d,
             "moe_inter": shape.I, "experts": shape.E, "top_k": shape.k, "shared_inter": shape.Is,
             "weights": "e4m3 + fp32 128x128 block scales" if shape.wtype == "fp8" else "bf16",
-            "activations": "e4m3 1x128 groups into the expert GEMMs" if shape.wtype == "fp8" else "bf16",
+            "activations": ("e4m3 1x128 groups into the expert GEMMs" if act8 else
+                            "bf16 (e4m3 weight tiles widened to bf16 on chip)") if shape.wtype == "fp8" else "bf16",
             "parallelism": "replicas (token data parallel, no collective)",
             "l2": "inputs larger than L2 (expert weights stream from HBM every step)"}
 
@@ -219,6 +220,9 @@ def run_ours(args, shape, rank, world, device):
     torch.cuda.set_device(device)
     inputs = make_inputs(shape, device)
     cfg = moe.Config.from_shape(shape)
+    act8 = args.act == "fp8" and shape.wtype == "fp8"
+    if shape.wtype == "fp8" and not act8:
+        cfg = dataclasses.replace(cfg, amode=moe.MOE_ACT_BF16)
     layer = moe.MoELayer(cfg, {n: v for n, v in inputs.items() if n not in ("x", "residual")}, device=device)
     x, r = inputs["x"], inputs["residual"]
     out = torch.empty_like(x)
@@ -321,8 +325,8 @@ def run_ours(args, shape, rank, world, device):
         return
 
     P, src = peaks()
-    wk = work(shape, counts)
-    fp8 = shape.wtype == "fp8"
+    wk = work(shape, counts, act8)
+    fp8 = act8             # FP8 tensor-core arithmetic
     tensor_peak = (2.0 if fp8 else 1.0) * P["bf16_tflops_sustained"]
     up_ms = float(stage[:, 4].mean())
     t_flop = wk["up_flops"] / (tensor_peak * 1e12) * 1e3
@@ -333,9 +337,10 @@ def run_ours(args, shape, rank, world, device):
     else:
         roof = {"bound": "hbm", "achieved": wk["up_bytes"] / (up_ms * 1e-3) / 1e9, "peak": P["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = recorded_traffic(shape.name, "gemm_up")
+    roof["traffic"] = recorded_traffic(shape.name, "gemm_up") if act8 or shape.wtype != "fp8" else None
     roof["algorithmic_bytes"] = wk["up_bytes"]
-    roof["kernel"] = "gemm_kernel up (w1|w3 + SwiGLU + FP8 quant of h)"
+    roof["kernel"] = ("gemm_kernel up (w1|w3 + SwiGLU + FP8 quant of h)" if act8 else
+                      "gemm_kernel up (w1|w3 + SwiGLU, bf16 operands)")
     roof["peak_source"] = (f"{src} MEASURED_PEAKS.json: " +
                            ("2 x bf16_tflops_sustained (fp8 dense = 2 x bf16)" if roof["bound"] == "tensor" and fp8 else
                             "bf16_tflops_sustained" if roof["bound"] == "tensor" else "hbm_gbs"))
@@ -346,7 +351,7 @@ def run_ours(args, shape, rank, world, device):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic (seeded counter-based generator)",
-        "config": config_block(shape),
+        "config": config_block(shape, act8),
         "roofline": roof,
         "step_roofline": {"tflops": wk["step_flops"] / (ms * 1e-3) / 1e12,
                           "tflops_frac_of_peak": wk["step_flops"] / (ms * 1e-3) / 1e12 / tensor_peak,
@@ -363,7 +368,7 @@ def run_ours(args, shape, rank, world, device):
         "clocks": clk,
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = oracle_throughput(shape, inputs, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = oracle_throughput(shape, inputs, budget_s=args.cpu_budget, act8=act8)
     print(json.dumps(line), flush=True)
 
 
@@ -378,6 +383,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--tokens", type=int, default=0, help="override T (smaller cases for profiling)")
     ap.add_argument("--experts", type=int, default=0, help="override E (smaller cases for profiling)")
+    ap.add_argument("--act", default="fp8", choices=["fp8", "bf16"],
+                    help="activations of the FP8-weight workloads: 1x128 FP8 (default) or bf16")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     shape = synthetic.CONFIGS[args.config]
