@@ -204,6 +204,19 @@ def run_reference(args, shape, rank):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(values, world, device="cpu"):
+    """Every rank's timings -> the slowest rank's, on every rank (one MAX all-reduce; no-op alone)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def whole_job_rate(tokens_per_rank, world, ms_per_step):
+    """Tokens/s of the whole job: all ranks' tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / (ms_per_step * 1e-3)
+
+
 def config_block(shape, act8=True):
     desc = synthetic.DESCRIPTIONS.get(shape.name, "reduced case of " + shape.name.split("-")[0] + " (profiling only)")
     return {"workload": f"{shape.name}: {desc}", "tokens": shape.T, "dim": shape.d,
@@ -317,10 +330,7 @@ def run_ours(args, shape, rank, world, device):
     if not torch.equal(oh[(ke - 1) & 1], out.cpu()):
         raise RuntimeError("end-to-end output differs from the device-resident run")
 
-    t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, device)
     if rank != 0:
         return
 
@@ -345,8 +355,7 @@ def run_ours(args, shape, rank, world, device):
                            ("2 x bf16_tflops_sustained (fp8 dense = 2 x bf16)" if roof["bound"] == "tensor" and fp8 else
                             "bf16_tflops_sustained" if roof["bound"] == "tensor" else "hbm_gbs"))
     roof["ms_per_launch"] = up_ms
-    tokens = shape.T * world
-    value = tokens / (ms * 1e-3)
+    value = whole_job_rate(shape.T, world, ms)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -360,7 +369,7 @@ def run_ours(args, shape, rank, world, device):
                           "touched_experts": wk["touched"]},
         "stage_ms": {n: float(stage[:, j].mean()) for j, n in enumerate(
             ["norm", "gate_gemm", "topk", "route", "gemm_up", "gemm_down", "combine"])},
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": 2 * x.numel() * 2,
+        "e2e": {"value": whole_job_rate(shape.T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": 2 * x.numel() * 2,
                 "d2h_bytes_per_step": 2 * x.numel() * 2, "ms_per_step": e2e_ms,
                 "how": "moe_forward on host buffers: per step H2D of x and residual, D2H of out and the new "
                        "residual (pinned), uploads / forwards / downloads pipelined on three streams"},
