@@ -34,22 +34,47 @@ __device__ __forceinline__ bool better64(double sa, int ea, double sb, int eb) {
     return sa > sb || (sa == sb && ea < eb);
 }
 
-// float64 dot product of the token's normed row with one router row, by the whole warp
-__device__ __forceinline__ double dot64(const uint4* __restrict__ xr, const uint4* __restrict__ wr, int nv, int lane) {
-    double acc = 0.0;
-    for (int v = lane; v < nv; v += 32) {
-        const uint4 a = xr[v], b = wr[v];
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+constexpr int kDotBatch = 8;   // router rows per pass over the token's row
+
+// float64 dot products of the token's normed row with up to kDotBatch router rows (ids in ex[0..nb),
+// warp-uniform), by the whole warp: one pass over the row, every row's loads of a step in flight
+// together.  bf16 x bf16 products are exact in float64; the sums are float64.
+__device__ __forceinline__ void dot64_batch(const uint4* __restrict__ xr, const uint16_t* __restrict__ gw, int d,
+                                            const int (&ex)[kDotBatch], int nb, int lane, double (&out)[kDotBatch]) {
+    const int nv = d >> 3;
+    double acc[kDotBatch];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            acc = fma(static_cast<double>(__uint_as_float(aw[i] << 16)), static_cast<double>(__uint_as_float(bw[i] << 16)), acc);
-            acc = fma(static_cast<double>(__uint_as_float(aw[i] & 0xFFFF0000u)),
-                      static_cast<double>(__uint_as_float(bw[i] & 0xFFFF0000u)), acc);
+    for (int i = 0; i < kDotBatch; ++i) acc[i] = 0.0;
+    for (int v = lane; v < nv; v += 32) {
+        const uint4 a = xr[v];
+        uint4 b[kDotBatch];
+#pragma unroll
+        for (int i = 0; i < kDotBatch; ++i)
+            if (i < nb) b[i] = reinterpret_cast<const uint4*>(gw + static_cast<size_t>(ex[i]) * d)[v];
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+        double ad[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            ad[2 * q] = static_cast<double>(__uint_as_float(aw[q] << 16));
+            ad[2 * q + 1] = static_cast<double>(__uint_as_float(aw[q] & 0xFFFF0000u));
+        }
+#pragma unroll
+        for (int i = 0; i < kDotBatch; ++i) {
+            if (i >= nb) continue;
+            const uint32_t bw[4] = {b[i].x, b[i].y, b[i].z, b[i].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                acc[i] = fma(ad[2 * q], static_cast<double>(__uint_as_float(bw[q] << 16)), acc[i]);
+                acc[i] = fma(ad[2 * q + 1], static_cast<double>(__uint_as_float(bw[q] & 0xFFFF0000u)), acc[i]);
+            }
         }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
-    return acc;
+    for (int i = 0; i < kDotBatch; ++i) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], off);
+        out[i] = acc[i];
+    }
 }
 
 __global__ void __launch_bounds__(kTopkWarps * 32)
@@ -111,19 +136,39 @@ topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, co
     if (redo) {
         // float64 scores of every member of S (each lane keeps its own experts' values), then the
         // top k inside S by float64 score, lower index first on equal scores
-        const int nv = d >> 3;
         const uint4* xr = reinterpret_cast<const uint4*>(xn + static_cast<size_t>(t) * d);
 #pragma unroll
+        for (int j = 0; j < J; ++j) s64[j] = -1.0;
+        // walk the members of S in expert order, kDotBatch router rows per pass over the row
+        int ex[kDotBatch];
+        int nb = 0;
         for (int j = 0; j < J; ++j) {
-            s64[j] = -1.0;
             uint32_t m = __ballot_sync(0xFFFFFFFFu, (S >> j) & 1u);
             while (m) {
                 const int src = __ffs(m) - 1;
                 m &= m - 1;
-                const int e = src + 32 * j;
-                double zz = dot64(xr, reinterpret_cast<const uint4*>(gw + static_cast<size_t>(e) * d), nv, lane);
-                if (bias) zz += static_cast<double>(bias[e]);
-                if (lane == src) s64[j] = 1.0 / (1.0 + exp(-zz));
+                ex[nb++] = src + 32 * j;
+                const bool last = !m && [&] {
+                    for (int jj = j + 1; jj < J; ++jj)
+                        if (__ballot_sync(0xFFFFFFFFu, (S >> jj) & 1u)) return false;
+                    return true;
+                }();
+                if (nb == kDotBatch || last) {
+                    double zz[kDotBatch];
+                    dot64_batch(xr, gw, d, ex, nb, lane, zz);
+#pragma unroll
+                    for (int i = 0; i < kDotBatch; ++i) {
+                        if (i >= nb) continue;
+                        const int e = ex[i];
+                        double z64 = zz[i];
+                        if (bias) z64 += static_cast<double>(bias[e]);
+                        const double sc = 1.0 / (1.0 + exp(-z64));
+#pragma unroll
+                        for (int jj = 0; jj < J; ++jj)
+                            if (e == lane + 32 * jj) s64[jj] = sc;
+                    }
+                    nb = 0;
+                }
             }
         }
         fin = 0u;

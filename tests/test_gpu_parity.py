@@ -155,3 +155,49 @@ def test_full_size_workloads(name, n_sample):
     print(name, json.dumps(report))
     if name == "C5":
         assert report["empty_experts"] >= 15
+
+
+def test_maximum_dim_8192():
+    """The largest d the library accepts (the norm holds a whole row in registers up to 8192)."""
+    shape = _shape(T=130, d=8192, I=1024, E=8, k=2, shared_inter=1024, seed=23)
+    _full_check(shape, inputs_for(shape), {})
+
+
+def test_single_expert_top1():
+    """E = 1, k = 1: the router always picks expert 0 with weight 1, so the layer is the textbook
+    SwiGLU MLP of that expert plus the shared one."""
+    shape = _shape(T=200, E=1, k=1, seed=24)
+    run, ref = _full_check(shape, inputs_for(shape), {})
+    assert np.all(run.idx == 0) and np.all(run.w == 1.0)
+
+
+@pytest.mark.parametrize("wtype", ["fp8", "bf16"])
+def test_zero_input_gives_zero_output(wtype):
+    """x = residual = 0: s = 0, xn = 0 (eps keeps the norm finite), every score is 0.5 (lowest
+    indices win), every quant scale is 1 with zero codes, and the output is exactly zero."""
+    shape = _shape(T=140, wtype=wtype, I=1024, seed=25)
+    inp = inputs_for(shape)
+    inp["x"] = torch.zeros_like(inp["x"])
+    inp["residual"] = torch.zeros_like(inp["residual"])
+    run, ref = _full_check(shape, inp, {}, strict=True)
+    assert not run.out.any() and not run.residual_out.any() and not run.xn.any()
+    assert np.all(np.sort(run.idx, 1) == np.arange(shape.k))
+
+
+def test_prefill_shape_with_ragged_token_count():
+    """The prefill layer shape (d 7168, 256 experts, top-8) at T = 4099: the last M tile of the shared
+    expert and of many experts is ragged; sampled tokens include the last one."""
+    shape = dataclasses.replace(synthetic.CONFIGS["C4"], name="C4-ragged", T=4099)
+    inp = inputs_for(shape)
+    run = GpuRun(shape, inp)
+    o = oracle.Oracle(shape, inp)
+    report = {}
+    route = o.forward(route_only=True)
+    allt = np.arange(shape.T, dtype=np.int32)
+    check_norm(run, route, allt, report)
+    check_routing(run, route, allt, report)
+    toks = sample_tokens(run, route, 24, seed=7)
+    assert shape.T - 1 in toks
+    ref = o.forward(toks)
+    check_out(run, ref, toks, report)
+    print(shape.name, json.dumps(report))
