@@ -411,7 +411,10 @@ void oracle_forward(const oracle_cfg* c, const oracle_inputs* in, int n, const i
 
         oracle_norm_token(d, in->x + (size_t)t * d, in->residual ? in->residual + (size_t)t * d : NULL,
                           in->norm_w, c->eps, xn, ro, xn64, NULL);
-        oracle_gate_token(d, E, k, xn, in->gate_w, in->gate_bias, scores, idx, w, &margin);
+        /* a dense block ("MoE update" page, Block excerpt: the first n_dense_layers blocks use the
+         * MLP instead of the MoE) has no router: E = 0, k = 0, and the MLP is the shared SwiGLU */
+        if (E > 0) oracle_gate_token(d, E, k, xn, in->gate_w, in->gate_bias, scores, idx, w, &margin);
+        else margin = INFINITY;
 
         if (!route_only) {
             /* the activation every expert sees: xn itself, or its FP8 quant */

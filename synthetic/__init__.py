@@ -74,6 +74,10 @@ CONFIGS = {
     "C4": MoEShape("C4", T=16384, d=7168, I=2048, E=256, k=8, n_shared=1, shared_inter=2048, wtype="fp8", seed=3),
     "C5": MoEShape("C5", T=8192, d=7168, I=2048, E=256, k=8, n_shared=1, shared_inter=2048, wtype="fp8", seed=4,
                    r_std=2.0, zipf_bias=True),
+    # a dense block: no router, one SwiGLU MLP (held as the "shared" weights).  The pages do not
+    # give the dense MLP's width; 9 x 2048 = 18432 gives it the per-token FLOPs of the MoE block
+    # (8 routed + 1 shared SwiGLU of 2048).
+    "D1": MoEShape("D1", T=16384, d=7168, I=128, E=0, k=0, n_shared=1, shared_inter=18432, wtype="fp8", seed=5),
 }
 
 DESCRIPTIONS = {
@@ -82,6 +86,7 @@ DESCRIPTIONS = {
     "C3": "DeepSeek-V3.2 MoE shape, decode batch: T=128, d=7168, inter=2048, 256 experts, top-8, 1 shared, FP8 128x128",
     "C4": "DeepSeek-V3.2 MoE shape, prefill batch: T=16384 (B=4 x 4096), d=7168, inter=2048, 256 experts, top-8, FP8",
     "C5": "DeepSeek-V3.2 MoE shape, Zipf(1.2) gate bias: T=8192, 256 experts, top-8, FP8, residual ~N(0,4)",
+    "D1": "dense-MLP block of the same model (no router): T=16384, d=7168, MLP inter 18432 (stand-in width), FP8",
 }
 
 
@@ -197,7 +202,7 @@ def generate(shape: MoEShape, device="cpu", alpha: Optional[float] = None, with_
     g["x"] = normal(sd, "x", (T, d), shape.x_std, device=device)
     g["residual"] = normal(sd, "residual", (T, d), shape.r_std, device=device)
     g["norm_w"] = torch.ones(d, dtype=torch.float32, device=device)
-    g["gate_w"] = normal(sd, "gate_w", (E, d), shape.gate_std, device=device)
+    g["gate_w"] = normal(sd, "gate_w", (E, d), shape.gate_std, device=device) if E > 0 else None
     if shape.zipf_bias:
         if alpha is None:
             raise ValueError("the Zipf-bias workload needs its alpha (tests/golden/c5_alpha.json)")
@@ -217,6 +222,14 @@ def generate(shape: MoEShape, device="cpu", alpha: Optional[float] = None, with_
     def scl(name, rows, cols):
         return _uniform_range(sd, name + ":scale", (rows // 128, cols // 128), 1e-4, 2e-3, device)
 
+    if E == 0:   # dense block: only the MLP ("shared") weights
+        g["sw1"], g["sw3"], g["sw2"] = mat("sw1", Is, d), mat("sw3", Is, d), mat("sw2", d, Is)
+        g["w1"] = g["w3"] = g["w2"] = g["s1"] = g["s3"] = g["s2"] = None
+        if fp8:
+            g["ss1"], g["ss3"], g["ss2"] = scl("sw1", Is, d), scl("sw3", Is, d), scl("sw2", d, Is)
+        else:
+            g["ss1"] = g["ss3"] = g["ss2"] = None
+        return g
     sel = range(E) if experts is None else experts
     w1 = torch.zeros(E, I, d, dtype=wdt, device=device)
     w3 = torch.zeros(E, I, d, dtype=wdt, device=device)

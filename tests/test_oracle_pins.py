@@ -359,3 +359,33 @@ def test_parameter_accounting_from_pages():
     assert round(gold["moe_params_per_block"] / 2 ** 30, 1) == gold["moe_fp8_gib_per_block_rounded"]
     s = synthetic.CONFIGS["C3"]
     assert (s.d, s.I, s.E, s.Is) == (d, I, E, I)
+
+
+@pytest.mark.parametrize("wtype", ["bf16", "fp8"])
+def test_dense_block_is_textbook_swiglu_and_matches_the_single_expert_route(wtype):
+    """A dense block ("MoE update" page, Block excerpt: MLP(dim, inter_dim) in the first blocks) has
+    no router: out = MLP(ffn_norm(x)).  Pinned to the SwiGLU evaluated here with torch matmuls, and
+    bit-for-bit to the routed path with one expert, top-1 (weight exactly 1) holding the same MLP."""
+    d, Is = 256, 384
+    dense = synthetic.MoEShape("pin-dense", T=24, d=d, I=128, E=0, k=0, n_shared=1, shared_inter=Is,
+                               wtype=wtype, seed=12)
+    inp = _layer(dense)
+    assert inp["gate_w"] is None and inp["w1"] is None
+    o = oracle.Oracle(dense, inp, act_fp8=False)
+    r = o.forward()
+    assert r["idx"].shape == (24, 0) and np.all(np.isinf(r["margin"]))
+    xn = _xn_all(o)
+    y = torch.stack([_textbook_swiglu(a, _w(inp["sw1"], inp["ss1"]), _w(inp["sw3"], inp["ss3"]),
+                                      _w(inp["sw2"], inp["ss2"])) for a in xn])
+    _close(torch.from_numpy(bf16_bits_to_f64(r["out"])), y, [y])
+    # the same MLP as the only routed expert, no shared expert, in both activation modes
+    routed = synthetic.MoEShape("pin-dense-routed", T=24, d=d, I=Is, E=1, k=1, n_shared=0, shared_inter=0,
+                                wtype=wtype, seed=12)
+    rin = dict(inp, gate_w=torch.zeros(1, d, dtype=torch.bfloat16), w1=inp["sw1"][None], w3=inp["sw3"][None],
+               w2=inp["sw2"][None], s1=None if inp["ss1"] is None else inp["ss1"][None],
+               s3=None if inp["ss3"] is None else inp["ss3"][None], s2=None if inp["ss2"] is None else inp["ss2"][None],
+               sw1=None, sw3=None, sw2=None, ss1=None, ss3=None, ss2=None)
+    for act8 in ([False, True] if wtype == "fp8" else [False]):
+        a = oracle.Oracle(dense, inp, act_fp8=act8).forward()
+        b = oracle.Oracle(routed, rin, act_fp8=act8).forward()
+        assert np.array_equal(a["out"], b["out"]) and np.array_equal(a["residual_out"], b["residual_out"])
