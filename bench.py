@@ -253,8 +253,9 @@ def run_ours(args, shape, rank, world, device):
     st = moe.moe_get_status(layer.workspace)
     if st != moe.MOE_OK:
         raise RuntimeError(moe.status_string(st))
-    counts = torch.empty(shape.E, dtype=torch.int32, device=device)
-    moe.moe_debug_routing(cfg, layer.workspace, counts=counts)
+    counts = torch.zeros(shape.E, dtype=torch.int32, device=device)
+    if shape.E > 0:                       # a dense block has no routing
+        moe.moe_debug_routing(cfg, layer.workspace, counts=counts)
     counts = counts.cpu().numpy()
 
     def barrier():

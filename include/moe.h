@@ -76,8 +76,11 @@ typedef struct {
     int32_t num_tokens;    /* T = B * S, >= 1 */
     int32_t dim;           /* d, multiple of 256, at most 8192 */
     int32_t inter_dim;     /* I (moe_inter_dim), multiple of 128 */
-    int32_t n_experts;     /* E routed experts, 1..256, multiple of 8 or E <= 8 */
-    int32_t top_k;         /* k, 1..E */
+    int32_t n_experts;     /* E routed experts, 1..256, multiple of 8 or E <= 8; 0 = a dense block
+                              ("MoE update" page, Block excerpt: MLP(dim, inter_dim) in the first
+                              n_dense_layers blocks): no router, the MLP given as the shared
+                              SwiGLU (shared_inter = its width), out = MLP(ffn_norm(x)) */
+    int32_t top_k;         /* k, 1..E; 0 for a dense block */
     int32_t shared_inter;  /* width of the shared SwiGLU (n_shared * per-expert inter; several
                               shared experts are one SwiGLU with concatenated hidden units);
                               multiple of 128; 0 = no shared expert */
@@ -106,9 +109,10 @@ size_t moe_workspace_bytes(const moe_config_t* cfg);
  *   x            [T, d] bf16            input of ffn_norm (the attention output)
  *   residual     [T, d] bf16 or NULL    residual stream; NULL = RMSNorm without the add
  *   norm_w       [d] float32            RMSNorm gain
- *   gate_w       [E, d] bf16            router weight
+ *   gate_w       [E, d] bf16            router weight (ignored, may be NULL, for a dense block)
  *   gate_bias    [E] float32 or NULL    per-expert bias added to the logits before the sigmoid
- *   w            expert weights (moe_weights_t)
+ *   w            expert weights (moe_weights_t); a dense block uses only sw1, sw3, sw2 (and
+ *                ss1, ss3, ss2 for FP8), the routed fields may be NULL
  *   out          [T, d] bf16            delta_ffn
  *   residual_out [T, d] bf16            new residual = bf16(x + residual); may equal residual
  *                                       (in place); unused when residual is NULL
@@ -144,7 +148,7 @@ moe_status_t moe_get_status(const void* workspace, void* stream);
  * used this workspace: idx [T, k] int32 (slot order = descending score), weights [T, k]
  * float32, counts [E] int32 (tokens per expert), near_tie [T] uint8 (1 = another expert was
  * within the candidate window of the k-th winner and the selection was re-decided in float64).
- * Any output pointer may be NULL. */
+ * Any output pointer may be NULL.  MOE_ERR_INVALID_ARG for a dense block (it has no routing). */
 moe_status_t moe_debug_routing(const moe_config_t* cfg, const void* workspace, int32_t* idx,
                                float* weights, int32_t* counts, uint8_t* near_tie, void* stream);
 
@@ -190,7 +194,9 @@ moe_status_t moe_route_noalloc(const int32_t* idx, int32_t num_tokens, int32_t t
 moe_status_t moe_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int64_t limit_cycles,
                                        void* stream);
 
-/* Number of kernel launches one moe_forward enqueues for this configuration. */
+/* Number of kernel launches one moe_forward enqueues for this configuration (10; 3 for a dense
+ * block: norm and the two SwiGLU GEMMs, the second writing out directly).  For a dense block the
+ * traced events 2-4 and 6-7 are recorded back to back (no router, no combine). */
 int32_t moe_launches_per_forward(const moe_config_t* cfg);
 
 /* Static description of a status code. */

@@ -87,8 +87,13 @@ bool encode_store_map_2d(CUtensorMap* map, const void* base, int elem_bytes, uin
 bool make_layout(const moe_config_t& c, Layout& L) {
     if (c.num_tokens < 1 || c.dim < 256 || c.dim % 256 || c.dim > 8192 || c.inter_dim < 128 || c.inter_dim % 128)
         return false;
-    if (c.n_experts < 1 || c.n_experts > kMaxExperts || (c.n_experts > 8 && c.n_experts % 8)) return false;
-    if (c.top_k < 1 || c.top_k > c.n_experts) return false;
+    if (c.n_experts == 0) {
+        // dense block: no router, the MLP is the shared SwiGLU
+        if (c.top_k != 0 || c.shared_inter < 128) return false;
+    } else {
+        if (c.n_experts < 1 || c.n_experts > kMaxExperts || (c.n_experts > 8 && c.n_experts % 8)) return false;
+        if (c.top_k < 1 || c.top_k > c.n_experts) return false;
+    }
     if (c.shared_inter < 0 || c.shared_inter % 128) return false;
     if (c.wtype != MOE_W_BF16 && c.wtype != MOE_W_FP8_E4M3_B128) return false;
     if (c.amode != MOE_ACT_FP8_1x128 && c.amode != MOE_ACT_BF16) return false;
@@ -101,6 +106,7 @@ bool make_layout(const moe_config_t& c, Layout& L) {
     L.k = c.top_k;
     L.Is = c.shared_inter;
     L.fp8 = c.wtype == MOE_W_FP8_E4M3_B128;
+    L.dense = c.n_experts == 0;
     L.act8 = L.fp8 && c.amode == MOE_ACT_FP8_1x128;
     L.Tpad = static_cast<int>(align_up(L.T, kBM));
     L.R = static_cast<int>(align_up(static_cast<size_t>(L.T) * L.k + static_cast<size_t>(L.E) * (kBM - 1), kBM));
@@ -119,7 +125,12 @@ bool make_layout(const moe_config_t& c, Layout& L) {
     L.xn = take(static_cast<size_t>(L.T) * L.d * 2);
     L.xq = take(L.act8 ? static_cast<size_t>(L.T) * L.d : 0);
     L.xs = take(L.act8 ? static_cast<size_t>(L.KBd) * L.Tpad * 4 : 0);
-    L.logits = take(static_cast<size_t>(L.T) * L.E * 4);
+    // few tokens leave the router GEMM with few tiles: split its K so that more SMs stream it
+    {
+        const int tiles = (L.T + kBM - 1) / kBM;
+        L.ksplit = tiles >= 64 ? 1 : std::min({16, 128 / tiles, L.d / 64});
+    }
+    L.logits = take(static_cast<size_t>(L.T) * L.E * 4 * L.ksplit);
     L.idx = take(static_cast<size_t>(L.T) * L.k * 4);
     L.w = take(static_cast<size_t>(L.T) * L.k * 4);
     L.flag = take(L.T);
@@ -139,7 +150,7 @@ bool make_layout(const moe_config_t& c, Layout& L) {
     L.h_sh = take(static_cast<size_t>(L.Tpad) * L.Is * ab);
     L.hs_sh = take(L.act8 ? static_cast<size_t>(L.KBs) * L.Tpad * 4 : 0);
     L.y = take(static_cast<size_t>(L.R) * L.d * 2);
-    L.y_sh = take(static_cast<size_t>(L.T) * L.d * 2);
+    L.y_sh = take(L.dense ? 0 : static_cast<size_t>(L.T) * L.d * 2);   // dense: the MLP writes out directly
     L.total = o;
     return true;
 }
@@ -172,7 +183,66 @@ extern "C" size_t moe_workspace_bytes(const moe_config_t* cfg) {
 extern "C" int32_t moe_launches_per_forward(const moe_config_t* cfg) {
     Layout L;
     if (check_config(cfg, L) != MOE_OK) return 0;
-    return 10;   // norm, gate GEMM, top-k, hist, scan, scatter, gather, up, down, combine
+    return L.dense ? 3 : 10;   // norm, gate GEMM, top-k, hist, scan, scatter, gather, up, down, combine
+}
+
+// A dense block's MLP ("MoE update" page, Block excerpt: MLP(dim, inter_dim) in the first blocks):
+// the two GEMMs of the SwiGLU over all T tokens as one group, the second writing the bf16 output
+// rows straight into `out` (there is nothing to combine).
+static cudaError_t dense_mlp(const Layout& L, const moe_weights_t* w, uint8_t* ws, void* out, int sms,
+                             cudaStream_t s, int part) {
+    const bool fp8 = L.fp8, act8 = L.act8, a16 = fp8 && !act8;
+    auto bmap = [&](CUtensorMap* mp, const void* base, uint64_t inner, uint64_t rows) {
+        return a16 ? encode_raw_map_2d(mp, base, inner, rows) : encode_map_2d(mp, base, fp8, inner, rows);
+    };
+    const int mtiles = (L.T + kBM - 1) / kBM;
+    if (part == 0) {   // h = silu(xn W1^T) * (xn W3^T)
+        TensorMaps m;
+        bool ok = encode_map_2d(&m.a_s, ws + (act8 ? L.xq : L.xn), act8, L.d, L.T) &&
+                  bmap(&m.b0_s, w->sw1, L.d, L.Is) && bmap(&m.b1_s, w->sw3, L.d, L.Is);
+        if (act8) ok = ok && encode_store_map_2d(&m.o_s, ws + L.h_sh, 1, L.Is, L.Tpad, 64);
+        else m.o_s = m.a_s;
+        if (!ok) return cudaErrorInvalidValue;
+        m.a_r = m.a_s, m.b0_r = m.b0_s, m.b1_r = m.b1_s, m.o_r = m.o_s;
+        GemmParams p{};
+        p.G = 1;
+        p.single_rows = L.T;
+        p.n_tiles_s = L.Is / 128;
+        p.kb_s = act8 ? L.d / 128 : L.d / 64;
+        p.as_s = reinterpret_cast<const float*>(ws + L.xs);
+        p.as_ld_s = L.Tpad;
+        p.bs0_s = w->ss1;
+        p.bs1_s = w->ss3;
+        p.bs_cols_s = L.d / 128;
+        p.out_s = ws + L.h_sh;
+        p.out_ld_s = L.Is;
+        p.outs_s = reinterpret_cast<float*>(ws + L.hs_sh);
+        p.outs_ld_s = L.Tpad;
+        p.status = reinterpret_cast<uint32_t*>(ws + L.status);
+        return launch_gemm(kModeUp, fp8, a16, m, p, std::min(mtiles * p.n_tiles_s, sms), s);
+    }
+    {   // out = h W2^T
+        TensorMaps m;
+        bool ok = encode_map_2d(&m.a_s, ws + L.h_sh, act8, L.Is, L.Tpad) && bmap(&m.b0_s, w->sw2, L.Is, L.d);
+        if (fp8) ok = ok && encode_store_map_2d(&m.o_s, out, 2, L.d, L.T, 16);
+        else m.o_s = m.a_s;
+        if (!ok) return cudaErrorInvalidValue;
+        m.b1_s = m.b0_s;
+        m.a_r = m.a_s, m.b0_r = m.b0_s, m.b1_r = m.b0_s, m.o_r = m.o_s;
+        GemmParams p{};
+        p.G = 1;
+        p.single_rows = L.T;
+        p.n_tiles_s = L.d / 256;
+        p.kb_s = act8 ? L.Is / 128 : L.Is / 64;
+        p.as_s = reinterpret_cast<const float*>(ws + L.hs_sh);
+        p.as_ld_s = L.Tpad;
+        p.bs0_s = p.bs1_s = w->ss2;
+        p.bs_cols_s = L.Is / 128;
+        p.out_s = out;
+        p.out_ld_s = L.d;
+        p.status = reinterpret_cast<uint32_t*>(ws + L.status);
+        return launch_gemm(kModeDown, fp8, a16, m, p, std::min(mtiles * p.n_tiles_s, sms), s);
+    }
 }
 
 static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const void* residual,
@@ -182,10 +252,12 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
     Layout L;
     moe_status_t st = check_config(cfg, L);
     if (st != MOE_OK) return st;
-    if (!x || !norm_w || !gate_w || !w || !out) return MOE_ERR_INVALID_ARG;
+    if (!x || !norm_w || !w || !out) return MOE_ERR_INVALID_ARG;
     if (residual && !residual_out) return MOE_ERR_INVALID_ARG;
-    if (!w->w1 || !w->w3 || !w->w2) return MOE_ERR_INVALID_ARG;
-    if (L.fp8 && (!w->s1 || !w->s3 || !w->s2)) return MOE_ERR_INVALID_ARG;
+    if (!L.dense) {
+        if (!gate_w || !w->w1 || !w->w3 || !w->w2) return MOE_ERR_INVALID_ARG;
+        if (L.fp8 && (!w->s1 || !w->s3 || !w->s2)) return MOE_ERR_INVALID_ARG;
+    }
     if (L.Is > 0) {
         if (!w->sw1 || !w->sw3 || !w->sw2) return MOE_ERR_INVALID_ARG;
         if (L.fp8 && (!w->ss1 || !w->ss3 || !w->ss2)) return MOE_ERR_INVALID_ARG;
@@ -217,6 +289,17 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
     // 1. ffn_norm (+ FP8 activation quant)
     MOE_TRY(launch_norm(L, x, residual, norm_w, cfg->eps, residual_out, ws, s));
     MOE_TRY(mark(1));
+    if (L.dense) {
+        MOE_TRY(mark(2));
+        MOE_TRY(mark(3));
+        MOE_TRY(mark(4));
+        MOE_TRY(dense_mlp(L, w, ws, out, sms, s, 0));
+        MOE_TRY(mark(5));
+        MOE_TRY(dense_mlp(L, w, ws, out, sms, s, 1));
+        MOE_TRY(mark(6));
+        MOE_TRY(mark(7));
+        return MOE_OK;
+    }
 
     // 2. router logits on the tensor cores: xn [T, d] x Wg [E, d]^T
     {
@@ -234,11 +317,14 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
         p.single_rows = L.T;
         p.n_tiles_s = 1;
         p.kb_s = L.d / 64;
+        p.ksplit = L.ksplit;
+        p.kb_chunk = (p.kb_s + L.ksplit - 1) / L.ksplit;
+        p.split_stride = static_cast<size_t>(L.T) * L.E * 4;
         p.out_s = ws + L.logits;
         p.out_ld_s = L.E;
         p.n_valid_cols = L.E;
         p.status = reinterpret_cast<uint32_t*>(ws + L.status);
-        const int tiles = (L.T + kBM - 1) / kBM;
+        const int tiles = (L.T + kBM - 1) / kBM * L.ksplit;
         MOE_TRY(launch_gemm(kModeLogits, false, false, m, p, std::min(tiles, sms), s));
     }
     MOE_TRY(mark(2));
@@ -326,8 +412,8 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
             m.a_s = m.a_r, m.b0_s = m.b0_r, m.b1_s = m.b0_r;
         }
         if (fp8) {
-            ok = ok && encode_store_map_2d(&m.o_r, ws + L.y, 2, L.d, L.R, 32);
-            if (L.Is > 0) ok = ok && encode_store_map_2d(&m.o_s, ws + L.y_sh, 2, L.d, L.T, 32);
+            ok = ok && encode_store_map_2d(&m.o_r, ws + L.y, 2, L.d, L.R, 16);
+            if (L.Is > 0) ok = ok && encode_store_map_2d(&m.o_s, ws + L.y_sh, 2, L.d, L.T, 16);
             else m.o_s = m.o_r;
         } else {
             m.o_r = m.a_r, m.o_s = m.a_r;
@@ -397,6 +483,7 @@ extern "C" moe_status_t moe_debug_routing(const moe_config_t* cfg, const void* w
     Layout L;
     moe_status_t st = check_config(cfg, L);
     if (st != MOE_OK) return st;
+    if (L.dense) return MOE_ERR_INVALID_ARG;   // a dense block has no routing
     if (!workspace) return MOE_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const uint8_t* ws = static_cast<const uint8_t*>(workspace);

@@ -24,6 +24,7 @@ namespace moe {
 namespace {
 
 constexpr int kTopkWarps = 8;
+constexpr int kMaxSplit = 16;   // K parts of the router-logits GEMM (the layout never makes more)
 constexpr float kCandDelta = 2e-3f;   // logit units; far above the float32 logit error
 
 __device__ __forceinline__ bool better(float za, int ea, float zb, int eb) {
@@ -78,7 +79,7 @@ __device__ __forceinline__ void dot64_batch(const uint4* __restrict__ xr, const 
 }
 
 __global__ void __launch_bounds__(kTopkWarps * 32)
-topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, const uint16_t* __restrict__ xn,
+topk_kernel(const float* __restrict__ logits, int ksplit, const float* __restrict__ bias, const uint16_t* __restrict__ xn,
             const uint16_t* __restrict__ gw, int T, int E, int k, int d, int* __restrict__ idx, float* __restrict__ wout,
             uint8_t* __restrict__ flag) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -92,7 +93,19 @@ topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, co
         const int e = lane + 32 * j;
         float v = -INFINITY;
         if (e < E) {
-            v = logits[static_cast<size_t>(t) * E + e];
+            if (ksplit == 1) {
+                v = logits[static_cast<size_t>(t) * E + e];
+            } else {
+                // K parts of the logits GEMM: all loads first, then the sum in a fixed order
+                float part[kMaxSplit];
+#pragma unroll
+                for (int sp = 0; sp < kMaxSplit; ++sp)
+                    if (sp < ksplit) part[sp] = logits[(static_cast<size_t>(sp) * T + t) * E + e];
+                v = part[0];
+#pragma unroll
+                for (int sp = 1; sp < kMaxSplit; ++sp)
+                    if (sp < ksplit) v = __fadd_rn(v, part[sp]);
+            }
             if (bias) v = __fadd_rn(v, bias[e]);
             if (v != v) v = -INFINITY;
             valid |= 1u << j;
@@ -226,7 +239,7 @@ topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, co
 cudaError_t launch_topk(const Layout& L, const void* gate_w, const float* gate_bias, uint8_t* ws, cudaStream_t s) {
     const int grid = (L.T + kTopkWarps - 1) / kTopkWarps;
     topk_kernel<<<grid, kTopkWarps * 32, 0, s>>>(
-        reinterpret_cast<const float*>(ws + L.logits), gate_bias, reinterpret_cast<const uint16_t*>(ws + L.xn),
+        reinterpret_cast<const float*>(ws + L.logits), L.ksplit, gate_bias, reinterpret_cast<const uint16_t*>(ws + L.xn),
         static_cast<const uint16_t*>(gate_w), L.T, L.E, L.k, L.d, reinterpret_cast<int*>(ws + L.idx),
         reinterpret_cast<float*>(ws + L.w), ws + L.flag);
     return cudaGetLastError();

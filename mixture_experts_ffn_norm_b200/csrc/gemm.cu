@@ -54,6 +54,7 @@ constexpr uint32_t kTmemCols = 512;
 
 struct Tile {
     int g, mt, nt, shared, a_row0, rows_valid, kb, b_row0;
+    int kb0, ks;   // first K stage and K part (split-K launches; 0 otherwise)
 };
 
 __device__ __forceinline__ void decode_tile(int t, const int* ts, const int* rb, const int* rc, const GemmParams& p,
@@ -68,12 +69,20 @@ __device__ __forceinline__ void decode_tile(int t, const int* ts, const int* rb,
     ti.shared = (p.single_rows > 0) || (p.has_shared && lo == p.G - 1);
     const int cnt = rc[lo];
     const int mtiles = (cnt + kBM - 1) / kBM;
-    const int local = t - ts[lo];
+    int local = t - ts[lo];
+    ti.ks = 0;
+    if (p.ksplit > 1) {                       // K part outermost, then N, then M
+        const int per = mtiles * p.n_tiles_s;
+        ti.ks = local / per;
+        local -= ti.ks * per;
+    }
     ti.nt = local / mtiles;
     ti.mt = local - ti.nt * mtiles;
     ti.a_row0 = rb[lo] + ti.mt * kBM;
     ti.rows_valid = min(kBM, cnt - ti.mt * kBM);
-    ti.kb = ti.shared ? p.kb_s : p.kb_r;
+    const int kbt = ti.shared ? p.kb_s : p.kb_r;
+    ti.kb0 = ti.ks * p.kb_chunk;
+    ti.kb = p.ksplit > 1 ? min(p.kb_chunk, kbt - ti.kb0) : kbt;
     const int nrows = (mode == kModeUp) ? 128 : 256;
     ti.b_row0 = (ti.shared ? 0 : lo * p.b_rows_per_expert) + ti.nt * nrows;
 }
@@ -159,7 +168,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
     if (p.single_rows > 0) {
         if (threadIdx.x == 0) {
             ts_sh[0] = 0;
-            ts_sh[1] = ((p.single_rows + kBM - 1) / kBM) * p.n_tiles_s;
+            ts_sh[1] = ((p.single_rows + kBM - 1) / kBM) * p.n_tiles_s * max(1, p.ksplit);
             rb_sh[0] = 0;
             rc_sh[0] = p.single_rows;
         }
@@ -230,7 +239,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                     uint8_t* sa = smem + stage * SB;
                     uint8_t* sb = sa + (kA16 ? kStageBytes : kStageBytesA);   // kA16: the raw e4m3 area
                     mbar_arrive_expect_tx(&full_bar[stage], kA16 ? kStageBytesA + kRawBytes : kStageBytes);
-                    const int kx = kb * KX;
+                    const int kx = (ti.kb0 + kb) * KX;
                     tma_load_2d(sa, ma, &full_bar[stage], kx, ti.a_row0);
                     tma_load_2d(sb, mb0, &full_bar[stage], kx, ti.b_row0);
                     tma_load_2d(sb + (kA16 ? kRawBytes / 2 : 128 * 128), mb1, &full_bar[stage], kx, b1_row);
@@ -440,7 +449,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                 if constexpr (kMode == kModeLogits) {
                     // router logits, float32, columns 128c .. 128c+127 that are < n_valid_cols
                     if (valid) {
-                        float* dst = reinterpret_cast<float*>(out + static_cast<size_t>(grow) * out_ld * 4) + 128 * c;
+                        float* dst = reinterpret_cast<float*>(out + static_cast<size_t>(ti.ks) * p.split_stride +
+                                                              static_cast<size_t>(grow) * out_ld * 4) + 128 * c;
                         const int ncol = min(128, p.n_valid_cols - 128 * c);
                         if ((p.n_valid_cols & 3) == 0) {        // rows 16-byte aligned: vector stores
 #pragma unroll
@@ -513,23 +523,25 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                         os[static_cast<size_t>(ti.nt) * os_ld + grow] = sc;
                     }
                 } else {
-                    // y rows (bf16): 4 chunks of 32 columns, each through this warp's staging rows and
-                    // one TMA store of 32 x 32 bf16
+                    // y rows (bf16): 8 chunks of 16 columns through the two 1 KB halves of this warp's
+                    // staging rows, one TMA store of 32 x 16 bf16 each; a half is refilled as soon as the
+                    // store two chunks back has read it, so the stores overlap the packing
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        if (lane == 0) bulk_wait_read();
+                    for (int ch = 0; ch < 8; ++ch) {
+                        uint8_t* half = ostage + (ch & 1) * (kOutStageBytes / 2);
+                        if (lane == 0) bulk_wait_read_but1();
                         __syncwarp();
-                        uint4* srow = reinterpret_cast<uint4*>(ostage + lane * 64);
+                        uint4* srow = reinterpret_cast<uint4*>(half + lane * 32);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float* a8 = accf + ch * 32 + 8 * i;
+                        for (int i = 0; i < 2; ++i) {
+                            const float* a8 = accf + ch * 16 + 8 * i;
                             srow[i] = make_uint4(pack2(a8[0], a8[1]), pack2(a8[2], a8[3]), pack2(a8[4], a8[5]),
                                                  pack2(a8[6], a8[7]));
                         }
                         fence_async_shared();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_store_2d(ti.shared ? &tm_o_s : &tm_o_r, ostage, ti.nt * 256 + 128 * c + 32 * ch,
+                            tma_store_2d(ti.shared ? &tm_o_s : &tm_o_r, half, ti.nt * 256 + 128 * c + 16 * ch,
                                          ti.a_row0 + q * 32);
                             bulk_commit();
                         }

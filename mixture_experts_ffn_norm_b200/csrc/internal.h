@@ -24,7 +24,9 @@ enum GemmMode : int { kModeLogits = 0, kModeUp = 1, kModeDown = 2 };
 // Byte offsets of every region of the caller's workspace.
 struct Layout {
     int T, d, I, E, k, Is, Tpad, R, KBd, KBi, KBs, nchunks;
+    int ksplit;                 // K parts of the router-logits GEMM (float32 partials, summed by top-k)
     bool fp8, act8;
+    bool dense;                 // E = 0: a dense block, the MLP held as the shared SwiGLU, no router
     size_t status, xn, xq, xs, logits, idx, w, flag, counts, offsets, row_base, row_count,
         ts_up, ts_down, chunk_hist, row_of, row_token, a_perm, as_perm, h, hs, h_sh, hs_sh, y, y_sh, total;
 };
@@ -57,6 +59,10 @@ struct GemmParams {
     float* outs_r; float* outs_s;
     int outs_ld_r, outs_ld_s;
     int n_valid_cols;           // logits: columns actually stored (E)
+    // split K (single-group launches only): part ks covers K stages [ks * kb_chunk, ...) and writes
+    // its float32 partial tile at out + ks * split_stride bytes
+    int ksplit, kb_chunk;
+    size_t split_stride;
     uint32_t* status;
 };
 

@@ -38,14 +38,15 @@ def test_workspace_sizes_and_invalid_configs():
     for s in synthetic.CONFIGS.values():
         cfg = moe.Config.from_shape(s)
         assert moe.workspace_bytes(cfg) > 0
-        assert moe.launches_per_forward(cfg) == 10
+        assert moe.launches_per_forward(cfg) == (3 if s.E == 0 else 10)   # a dense block: norm + 2 GEMMs
     c4 = moe.Config.from_shape(synthetic.CONFIGS["C4"])
     assert moe.workspace_bytes(c4) < 8 * 2 ** 30
     # bf16 activations with FP8 weights: the permuted rows and h are 2 bytes wide, no activation scales
     c4_a16 = dataclasses.replace(c4, amode=moe.MOE_ACT_BF16)
     assert moe.workspace_bytes(c4) < moe.workspace_bytes(c4_a16) < 2 * moe.workspace_bytes(c4)
     bad = [dict(dim=200), dict(inter_dim=100), dict(top_k=0), dict(top_k=300), dict(n_experts=300),
-           dict(n_experts=12), dict(num_tokens=0), dict(shared_inter=64), dict(wtype=7)]
+           dict(n_experts=12), dict(num_tokens=0), dict(shared_inter=64), dict(wtype=7),
+           dict(n_experts=0), dict(n_experts=0, top_k=0, shared_inter=0)]   # dense: k = 0 and an MLP
     for b in bad:
         kw = dict(num_tokens=64, dim=256, inter_dim=128, n_experts=8, top_k=2, shared_inter=128,
                   wtype=moe.MOE_W_BF16, amode=moe.MOE_ACT_BF16)
