@@ -129,7 +129,7 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* res
  *   events[0] before the first launch      events[4] after the permutation kernels
  *   events[1] after the norm kernel        events[5] after the grouped GEMM up (w1|w3, SwiGLU)
  *   events[2] after the gate GEMM          events[6] after the grouped GEMM down (w2)
- *   events[3] after the top-k kernel       events[7] after the combine kernel
+ *   events[3] after the top-k kernels      events[7] after the combine kernel
  * n_events may be smaller than 8 (the later boundaries are then not recorded); NULL entries are
  * skipped.  Same arguments, errors and ownership as moe_forward otherwise. */
 moe_status_t moe_forward_traced(const moe_config_t* cfg, const void* x, const void* residual,
@@ -194,7 +194,7 @@ moe_status_t moe_route_noalloc(const int32_t* idx, int32_t num_tokens, int32_t t
 moe_status_t moe_selftest_wait_timeout(void* workspace, size_t workspace_bytes, int64_t limit_cycles,
                                        void* stream);
 
-/* Number of kernel launches one moe_forward enqueues for this configuration (10; 3 for a dense
+/* Number of kernel launches one moe_forward enqueues for this configuration (11; 3 for a dense
  * block: norm and the two SwiGLU GEMMs, the second writing out directly).  For a dense block the
  * traced events 2-4 and 6-7 are recorded back to back (no router, no combine). */
 int32_t moe_launches_per_forward(const moe_config_t* cfg);

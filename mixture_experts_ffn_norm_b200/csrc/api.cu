@@ -134,6 +134,7 @@ bool make_layout(const moe_config_t& c, Layout& L) {
     L.idx = take(static_cast<size_t>(L.T) * L.k * 4);
     L.w = take(static_cast<size_t>(L.T) * L.k * 4);
     L.flag = take(L.T);
+    L.redo = take(static_cast<size_t>(L.T) * 4);     // tokens listed for the float64 re-decision
     L.counts = take(static_cast<size_t>(L.E) * 4);
     L.offsets = take(static_cast<size_t>(L.E + 1) * 4);
     L.row_base = take(static_cast<size_t>(L.E + 1) * 4);
@@ -183,7 +184,7 @@ extern "C" size_t moe_workspace_bytes(const moe_config_t* cfg) {
 extern "C" int32_t moe_launches_per_forward(const moe_config_t* cfg) {
     Layout L;
     if (check_config(cfg, L) != MOE_OK) return 0;
-    return L.dense ? 3 : 10;   // norm, gate GEMM, top-k, hist, scan, scatter, gather, up, down, combine
+    return L.dense ? 3 : 11;   // norm, gate GEMM, top-k (2), hist, scan, scatter, gather, up, down, combine
 }
 
 // A dense block's MLP ("MoE update" page, Block excerpt: MLP(dim, inter_dim) in the first blocks):

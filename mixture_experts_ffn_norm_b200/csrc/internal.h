@@ -28,7 +28,7 @@ struct Layout {
     bool fp8, act8;
     bool dense;                 // E = 0: a dense block, the MLP held as the shared SwiGLU, no router
     size_t status, xn, xq, xs, logits, idx, w, flag, counts, offsets, row_base, row_count,
-        ts_up, ts_down, chunk_hist, row_of, row_token, a_perm, as_perm, h, hs, h_sh, hs_sh, y, y_sh, total;
+        ts_up, ts_down, chunk_hist, row_of, row_token, redo, a_perm, as_perm, h, hs, h_sh, hs_sh, y, y_sh, total;
 };
 
 bool make_layout(const moe_config_t& c, Layout& L);

@@ -20,6 +20,7 @@ namespace moe {
 namespace {
 
 constexpr int kRouteThreads = 256;
+constexpr int kMaxTopkGather = 8;   // top-k slots the gather keeps in registers
 
 __global__ void __launch_bounds__(kRouteThreads)
 hist_kernel(const int* __restrict__ idx, int N, int E, int* __restrict__ chunk_hist, uint32_t* status) {
@@ -136,21 +137,34 @@ scatter_kernel(const int* __restrict__ idx, int N, int E, int k, const int* __re
     }
 }
 
-// One warp per permuted row: copy the token's activation row and its group scales.
+// One warp per token: its activation row is read once and written to each of its k permuted rows
+// (row_of), with its group scales.  Walking tokens rather than destination rows keeps the source
+// row from being re-read k times -- with k rows' worth of writes streaming through L2 those re-reads
+// would come back from DRAM.
 __global__ void __launch_bounds__(kRouteThreads)
-gather_kernel(const int* __restrict__ row_token, const int* __restrict__ offsets, int E,
-              const uint4* __restrict__ src, int row_vecs, uint4* __restrict__ dst, const float* __restrict__ xs,
-              int Tpad, float* __restrict__ as, int R, int KB) {
-    const int total = offsets[E];
+gather_kernel(const int* __restrict__ row_of, int T, int k, const uint4* __restrict__ src, int row_vecs,
+              uint4* __restrict__ dst, const float* __restrict__ xs, int Tpad, float* __restrict__ as, int R, int KB) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int p = blockIdx.x * (kRouteThreads / 32) + warp; p < total; p += gridDim.x * (kRouteThreads / 32)) {
-        const int t = row_token[p];
-        if (t < 0) continue;
-        const uint4* s = src + static_cast<size_t>(t) * row_vecs;
-        uint4* d = dst + static_cast<size_t>(p) * row_vecs;
-        for (int v = lane; v < row_vecs; v += 32) d[v] = s[v];
+    for (int t = blockIdx.x * (kRouteThreads / 32) + warp; t < T; t += gridDim.x * (kRouteThreads / 32)) {
+        int rows[kMaxTopkGather];
+        const int kk = min(k, kMaxTopkGather);
+#pragma unroll
+        for (int j = 0; j < kMaxTopkGather; ++j) rows[j] = j < kk ? row_of[static_cast<size_t>(t) * k + j] : 0;
+        const uint4* sr = src + static_cast<size_t>(t) * row_vecs;
+#pragma unroll 2
+        for (int v = lane; v < row_vecs; v += 32) {
+            const uint4 val = sr[v];
+#pragma unroll
+            for (int j = 0; j < kMaxTopkGather; ++j)
+                if (j < kk) dst[static_cast<size_t>(rows[j]) * row_vecs + v] = val;
+            for (int j = kMaxTopkGather; j < k; ++j)          // wider top-k than the register list
+                dst[static_cast<size_t>(row_of[static_cast<size_t>(t) * k + j]) * row_vecs + v] = val;
+        }
         if (as)
-            for (int kb = lane; kb < KB; kb += 32) as[static_cast<size_t>(kb) * R + p] = xs[static_cast<size_t>(kb) * Tpad + t];
+            for (int kb = lane; kb < KB; kb += 32) {
+                const float sc = xs[static_cast<size_t>(kb) * Tpad + t];
+                for (int j = 0; j < k; ++j) as[static_cast<size_t>(kb) * R + row_of[static_cast<size_t>(t) * k + j]] = sc;
+            }
     }
 }
 
@@ -173,7 +187,7 @@ cudaError_t launch_route(const Layout& L, int ntu_r, int ntu_s, int ntd_r, int n
     const int row_bytes = L.act8 ? L.d : 2 * L.d;
     const int grid = 4 * num_sms();
     gather_kernel<<<grid, kRouteThreads, 0, s>>>(
-        reinterpret_cast<const int*>(ws + L.row_token), reinterpret_cast<const int*>(ws + L.offsets), L.E,
+        reinterpret_cast<const int*>(ws + L.row_of), L.T, L.k,
         reinterpret_cast<const uint4*>(ws + (L.act8 ? L.xq : L.xn)), row_bytes / 16,
         reinterpret_cast<uint4*>(ws + L.a_perm), L.act8 ? reinterpret_cast<const float*>(ws + L.xs) : nullptr,
         L.Tpad, L.act8 ? reinterpret_cast<float*>(ws + L.as_perm) : nullptr, L.R, L.KBd);
