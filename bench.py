@@ -331,7 +331,31 @@ def run_ours(args, shape, rank, world, device):
     if not torch.equal(oh[(ke - 1) & 1], out.cpu()):
         raise RuntimeError("end-to-end output differs from the device-resident run")
 
-    ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, device)
+    # optional: the same layer through moe_forward_next_norm (the next block's attn_norm fused into
+    # the combine; the update itself is not written)
+    nn_ms = None
+    if args.next_norm and shape.E > 0:
+        t_ = layer.t
+        g_next = (1.0 + synthetic.normal(shape.seed, "next_norm_w", (shape.d,), 0.1, device=device).float()).contiguous()
+        xn_next, r_next = torch.empty_like(x), torch.empty_like(x)
+        call = lambda: moe.moe_forward_next_norm(cfg, x, r, t_["norm_w"], t_["gate_w"], t_.get("gate_bias"),
+                                                 layer.wstruct, g_next, None, xn_next, r_next, layer.workspace)
+        for _ in range(W):
+            call()
+        torch.cuda.synchronize()
+        barrier()
+        n0, n1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n0.record(stream)
+        for _ in range(K):
+            call()
+        n1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        nn_ms = n0.elapsed_time(n1) / K
+        if moe.moe_get_status(layer.workspace) != moe.MOE_OK:
+            raise RuntimeError("moe_forward_next_norm failed")
+
+    ms, e2e_ms, nn_ms = max_over_ranks([ms, e2e_ms, -1.0 if nn_ms is None else nn_ms], world, device)
     if rank != 0:
         return
 
@@ -377,6 +401,13 @@ def run_ours(args, shape, rank, world, device):
         "gpu_launches": moe.launches_per_forward(cfg) * K,
         "clocks": clk,
     }
+    if nn_ms is not None and nn_ms > 0:
+        line["next_norm_fused"] = {
+            "ms_per_step": nn_ms, "tokens_per_s": whole_job_rate(shape.T, world, nn_ms),
+            "plain_ms_per_step": ms,
+            "how": "moe_forward_next_norm: the same layer with the next block's attn_norm in the combine; "
+                   "the update is not written (saves its write and the separate norm's read of it, "
+                   f"{2 * x.numel() * 2 / 1e6:.0f} MB per step)"}
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_throughput(shape, inputs, budget_s=args.cpu_budget, act8=act8)
     print(json.dumps(line), flush=True)
@@ -393,6 +424,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--tokens", type=int, default=0, help="override T (smaller cases for profiling)")
     ap.add_argument("--experts", type=int, default=0, help="override E (smaller cases for profiling)")
+    ap.add_argument("--next-norm", action="store_true",
+                    help="also time moe_forward_next_norm (the next block's attn_norm fused into the combine)")
     ap.add_argument("--act", default="fp8", choices=["fp8", "bf16"],
                     help="activations of the FP8-weight workloads: 1x128 FP8 (default) or bf16")
     args = ap.parse_args()

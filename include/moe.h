@@ -124,6 +124,27 @@ moe_status_t moe_forward(const moe_config_t* cfg, const void* x, const void* res
                          const moe_weights_t* w, void* out, void* residual_out,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* moe_forward with the next block's attn_norm fused into the combine ("MoE update" page, Block
+ * excerpt: residual additions happen inside the next normalisation, `x, residual =
+ * self.attn_norm(x, residual)` right after `x = self.ffn(x)`; RMSNorm excerpt for the arithmetic).
+ * Runs this layer exactly as moe_forward, then per token
+ *   s = fp32(delta) + fp32(bf16(x + residual))     delta = the MoE update (moe_forward's out)
+ *   next_residual = bf16(s)
+ *   next_xn = bf16(next_norm_w * (s * rsqrt(mean(s^2) + eps)))   (same arithmetic as ffn_norm)
+ * without writing delta to memory unless `out` is given.
+ *   residual       [T, d] bf16, required (the block's ffn_norm always adds one)
+ *   next_norm_w    [d] float32            the next block's attn_norm gain
+ *   out            [T, d] bf16 or NULL    delta, as moe_forward would write it
+ *   next_xn        [T, d] bf16            the next block's normed input
+ *   next_residual  [T, d] bf16            the next block's residual; may equal residual (in place)
+ * MOE_ERR_UNSUPPORTED for a dense block (n_experts = 0); other arguments, errors and ownership as
+ * moe_forward.  No counterpart call on the pages: it fuses two of their calls. */
+moe_status_t moe_forward_next_norm(const moe_config_t* cfg, const void* x, const void* residual,
+                                   const float* norm_w, const void* gate_w, const float* gate_bias,
+                                   const moe_weights_t* w, const float* next_norm_w, void* out,
+                                   void* next_xn, void* next_residual, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
 /* moe_forward that also records caller-created CUDA events (cudaEvent_t passed as void*) on
  * `stream` at the stage boundaries, for timing individual kernels inside a running workload:
  *   events[0] before the first launch      events[4] after the permutation kernels

@@ -19,7 +19,8 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
 MOE_W_BF16, MOE_W_FP8_E4M3_B128 = 0, 1
 MOE_ACT_FP8_1x128, MOE_ACT_BF16 = 0, 1
 
-EXPORTS = ("moe_workspace_bytes", "moe_forward", "moe_forward_traced", "moe_get_status", "moe_debug_routing",
+EXPORTS = ("moe_workspace_bytes", "moe_forward", "moe_forward_traced", "moe_forward_next_norm", "moe_get_status",
+           "moe_debug_routing",
            "moe_debug_norm", "moe_route_noalloc", "moe_selftest_wait_timeout", "moe_launches_per_forward",
            "moe_status_string")
 
@@ -58,6 +59,9 @@ def lib() -> C.CDLL:
         L.moe_forward_traced.restype = C.c_int
         L.moe_forward_traced.argtypes = [cfgp, vp, vp, vp, vp, vp, C.POINTER(moe_weights_t), vp, vp, vp, C.c_size_t,
                                          vp, C.POINTER(C.c_void_p), C.c_int32]
+        L.moe_forward_next_norm.restype = C.c_int
+        L.moe_forward_next_norm.argtypes = [cfgp, vp, vp, vp, vp, vp, C.POINTER(moe_weights_t), vp, vp, vp, vp, vp,
+                                            C.c_size_t, vp]
         L.moe_get_status.restype = C.c_int
         L.moe_get_status.argtypes = [vp, vp]
         L.moe_debug_routing.restype = C.c_int
@@ -151,6 +155,20 @@ def moe_forward_traced(cfg: Config, x, residual, norm_w, gate_w, gate_bias, weig
                                   workspace.numel() * workspace.element_size(), _stream(stream), arr, len(events))
     if check and rc != MOE_OK:
         raise MoeError(rc, "moe_forward_traced")
+    return rc
+
+
+def moe_forward_next_norm(cfg: Config, x, residual, norm_w, gate_w, gate_bias, weights, next_norm_w, out, next_xn,
+                          next_residual, workspace, stream=None, check=True) -> int:
+    """The forward pass with the next block's attn_norm fused in (see moe_forward_next_norm in
+    include/moe.h); ``out`` may be None."""
+    ws = weights if isinstance(weights, moe_weights_t) else weights_struct(weights)
+    rc = lib().moe_forward_next_norm(C.byref(cfg.c()), _ptr(x), _ptr(residual), _ptr(norm_w), _ptr(gate_w),
+                                     _ptr(gate_bias), C.byref(ws), _ptr(next_norm_w), _ptr(out), _ptr(next_xn),
+                                     _ptr(next_residual), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream))
+    if check and rc != MOE_OK:
+        raise MoeError(rc, "moe_forward_next_norm")
     return rc
 
 

@@ -249,11 +249,18 @@ static cudaError_t dense_mlp(const Layout& L, const moe_weights_t* w, uint8_t* w
 static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const void* residual,
                                  const float* norm_w, const void* gate_w, const float* gate_bias,
                                  const moe_weights_t* w, void* out, void* residual_out, void* workspace,
-                                 size_t workspace_bytes, void* stream_, void* const* events, int n_events) {
+                                 size_t workspace_bytes, void* stream_, void* const* events, int n_events,
+                                 const float* next_norm_w = nullptr, void* next_xn = nullptr) {
     Layout L;
     moe_status_t st = check_config(cfg, L);
     if (st != MOE_OK) return st;
-    if (!x || !norm_w || !w || !out) return MOE_ERR_INVALID_ARG;
+    const bool next = next_xn != nullptr;   // the next block's attn_norm fused into the combine
+    if (next && L.dense) return MOE_ERR_UNSUPPORTED;
+    if (next && (!next_norm_w || !residual || !residual_out)) return MOE_ERR_INVALID_ARG;
+    if (next && (next_xn == x || next_xn == residual || next_xn == out || next_xn == residual_out ||
+                 !aligned16(next_xn) || !aligned16(next_norm_w)))
+        return MOE_ERR_INVALID_ARG;
+    if (!x || !norm_w || !w || (!out && !next)) return MOE_ERR_INVALID_ARG;
     if (residual && !residual_out) return MOE_ERR_INVALID_ARG;
     if (!L.dense) {
         if (!gate_w || !w->w1 || !w->w3 || !w->w2) return MOE_ERR_INVALID_ARG;
@@ -269,7 +276,7 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
         if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
     if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return MOE_ERR_WORKSPACE;
-    if (out == x || out == residual || (residual_out && (residual_out == x || residual_out == out)))
+    if ((out && (out == x || out == residual)) || (residual_out && (residual_out == x || residual_out == out)))
         return MOE_ERR_INVALID_ARG;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream_);
@@ -447,7 +454,10 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
     }
     MOE_TRY(mark(6));
     // 7. weighted combine + shared add -> out
-    MOE_TRY(launch_combine(L, out, ws, s));
+    if (next)
+        MOE_TRY(launch_combine_next_norm(L, out, next_norm_w, cfg->eps, residual_out, next_xn, ws, s));
+    else
+        MOE_TRY(launch_combine(L, out, ws, s));
     MOE_TRY(mark(7));
     return MOE_OK;
 }
@@ -458,6 +468,16 @@ extern "C" moe_status_t moe_forward(const moe_config_t* cfg, const void* x, cons
                                     size_t workspace_bytes, void* stream) {
     return forward_impl(cfg, x, residual, norm_w, gate_w, gate_bias, w, out, residual_out, workspace,
                         workspace_bytes, stream, nullptr, 0);
+}
+
+extern "C" moe_status_t moe_forward_next_norm(const moe_config_t* cfg, const void* x, const void* residual,
+                                              const float* norm_w, const void* gate_w, const float* gate_bias,
+                                              const moe_weights_t* w, const float* next_norm_w, void* out,
+                                              void* next_xn, void* next_residual, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+    if (!next_xn) return MOE_ERR_INVALID_ARG;
+    return forward_impl(cfg, x, residual, norm_w, gate_w, gate_bias, w, out, next_residual, workspace,
+                        workspace_bytes, stream, nullptr, 0, next_norm_w, next_xn);
 }
 
 extern "C" moe_status_t moe_forward_traced(const moe_config_t* cfg, const void* x, const void* residual,

@@ -89,6 +89,10 @@ cudaError_t launch_topk(const Layout& L, const void* gate_w, const float* gate_b
 cudaError_t launch_route(const Layout& L, int ntu_r, int ntu_s, int ntd_r, int ntd_s, uint8_t* ws,
                          cudaStream_t s);
 cudaError_t launch_combine(const Layout& L, void* out, uint8_t* ws, cudaStream_t s);
+// the combine with the next block's RMSNorm: resid holds the block's new residual on entry and the
+// next residual on exit; out (the MoE update) may be NULL
+cudaError_t launch_combine_next_norm(const Layout& L, void* out, const float* gain, float eps, void* resid,
+                                     void* xn_next, uint8_t* ws, cudaStream_t s);
 
 int num_sms();
 

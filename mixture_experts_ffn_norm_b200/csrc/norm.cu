@@ -30,20 +30,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     return lo | (hi << 16);
 }
 
-// error-free sum of two doubles: (s, e) with s + e == a + b exactly
-__device__ __forceinline__ void two_sum(double a, double b, double& s, double& e) {
-    s = __dadd_rn(a, b);
-    const double bb = __dsub_rn(s, a);
-    e = __dadd_rn(__dsub_rn(a, __dsub_rn(s, bb)), __dsub_rn(b, bb));
-}
-
-__device__ __forceinline__ void dd_add(double& hi, double& lo, double hi2, double lo2) {
-    double s, e;
-    two_sum(hi, hi2, s, e);
-    hi = s;
-    lo = __dadd_rn(lo, __dadd_rn(lo2, e));
-}
-
 constexpr int kNormThreads = 128;
 constexpr int kMaxVec = 8;          // 16-byte vectors per thread: d <= 128 * 8 * 8 = 8192
 

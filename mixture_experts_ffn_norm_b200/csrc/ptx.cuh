@@ -272,4 +272,19 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// error-free sum of two doubles: (s, e) with s + e == a + b exactly (TwoSum)
+__device__ __forceinline__ void two_sum(double a, double b, double& s, double& e) {
+    s = __dadd_rn(a, b);
+    const double bb = __dsub_rn(s, a);
+    e = __dadd_rn(__dsub_rn(a, __dsub_rn(s, bb)), __dsub_rn(b, bb));
+}
+
+// (hi, lo) += (hi2, lo2), double-double
+__device__ __forceinline__ void dd_add(double& hi, double& lo, double hi2, double lo2) {
+    double s, e;
+    two_sum(hi, hi2, s, e);
+    hi = s;
+    lo = __dadd_rn(lo, __dadd_rn(lo2, e));
+}
+
 }  // namespace moe

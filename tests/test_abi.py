@@ -78,4 +78,13 @@ def test_forward_rejects_bad_arguments_without_touching_the_device():
     # bf16 weights with FP8 activations is not a mode
     bf16_a8 = moe.Config(64, 256, 128, 8, 2, 128, moe.MOE_W_BF16, moe.MOE_ACT_FP8_1x128).c()
     assert L.moe_forward(*args(cfg=bf16_a8)) == moe.MOE_ERR_INVALID_ARG
+    # the fused next-norm entry point: needs next_xn, a residual and the next gain; not for dense blocks
+    nn = lambda cfg=cfg, r=fake, g=fake + 12288, xn=fake + 16384: L.moe_forward_next_norm(
+        C.byref(cfg), fake, r, fake, fake, None, C.byref(w), g, None, xn, fake + 8192, fake, need, None)
+    assert nn(xn=None) == moe.MOE_ERR_INVALID_ARG
+    assert nn(r=None) == moe.MOE_ERR_INVALID_ARG
+    assert nn(g=None) == moe.MOE_ERR_INVALID_ARG
+    assert nn(xn=fake) == moe.MOE_ERR_INVALID_ARG                                # aliases x
+    dense = moe.Config(64, 256, 128, 0, 0, 256, moe.MOE_W_BF16, moe.MOE_ACT_BF16).c()
+    assert nn(cfg=dense) == moe.MOE_ERR_UNSUPPORTED
     assert moe.status_string(moe.MOE_ERR_WORKSPACE) == "workspace missing or too small"
