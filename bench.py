@@ -331,6 +331,30 @@ def run_ours(args, shape, rank, world, device):
     if not torch.equal(oh[(ke - 1) & 1], out.cpu()):
         raise RuntimeError("end-to-end output differs from the device-resident run")
 
+    # optional: the same forward captured once into a CUDA graph and replayed (one graph launch per step)
+    graph_ms = None
+    if args.graph:
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=side):
+            layer.forward(x, r, out, ro)
+        for _ in range(W):
+            graph.replay()
+        torch.cuda.synchronize()
+        barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(K):
+            graph.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        graph_ms = g0.elapsed_time(g1) / K
+        del graph
+        if moe.moe_get_status(layer.workspace) != moe.MOE_OK:
+            raise RuntimeError("graph replay failed")
+
     # optional: the same layer through moe_forward_next_norm (the next block's attn_norm fused into
     # the combine; the update itself is not written)
     nn_ms = None
@@ -355,7 +379,8 @@ def run_ours(args, shape, rank, world, device):
         if moe.moe_get_status(layer.workspace) != moe.MOE_OK:
             raise RuntimeError("moe_forward_next_norm failed")
 
-    ms, e2e_ms, nn_ms = max_over_ranks([ms, e2e_ms, -1.0 if nn_ms is None else nn_ms], world, device)
+    ms, e2e_ms, nn_ms, graph_ms = max_over_ranks(
+        [ms, e2e_ms, -1.0 if nn_ms is None else nn_ms, -1.0 if graph_ms is None else graph_ms], world, device)
     if rank != 0:
         return
 
@@ -401,6 +426,10 @@ def run_ours(args, shape, rank, world, device):
         "gpu_launches": moe.launches_per_forward(cfg) * K,
         "clocks": clk,
     }
+    if graph_ms is not None and graph_ms > 0:
+        line["cuda_graph"] = {"ms_per_step": graph_ms, "tokens_per_s": whole_job_rate(shape.T, world, graph_ms),
+                              "how": "the forward captured once with torch.cuda.graph and replayed; one graph launch "
+                                     "per step instead of the per-kernel launches"}
     if nn_ms is not None and nn_ms > 0:
         line["next_norm_fused"] = {
             "ms_per_step": nn_ms, "tokens_per_s": whole_job_rate(shape.T, world, nn_ms),
@@ -424,6 +453,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--tokens", type=int, default=0, help="override T (smaller cases for profiling)")
     ap.add_argument("--experts", type=int, default=0, help="override E (smaller cases for profiling)")
+    ap.add_argument("--graph", action="store_true", help="also time the forward replayed from a CUDA graph")
     ap.add_argument("--next-norm", action="store_true",
                     help="also time moe_forward_next_norm (the next block's attn_norm fused into the combine)")
     ap.add_argument("--act", default="fp8", choices=["fp8", "bf16"],

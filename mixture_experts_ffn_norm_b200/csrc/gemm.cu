@@ -34,6 +34,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include <mutex>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -611,9 +613,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
 template <bool kFp8, int kMode, bool kA16 = false>
 cudaError_t launch_one(const TensorMaps& m, const GemmParams& p, int grid, cudaStream_t s) {
     constexpr int smem = kA16 ? kSmemBytesA16 : kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<kFp8, kMode, kA16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
-    if (e != cudaSuccess) return e;
+    // the shared-memory opt-in is set once per device, so that a forward enqueued during stream
+    // capture (a CUDA graph) makes no call besides the launch
+    {
+        static std::mutex mu;
+        static bool done[64] = {};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev < 0 || dev >= 64 || !done[dev]) {
+            e = cudaFuncSetAttribute(gemm_kernel<kFp8, kMode, kA16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < 64) done[dev] = true;
+        }
+    }
     gemm_kernel<kFp8, kMode, kA16><<<grid, kGemmThreads, smem, s>>>(m.a_r, m.a_s, m.b0_r, m.b1_r, m.b0_s, m.b1_s,
                                                                     m.o_r, m.o_s, p);
     return cudaGetLastError();
