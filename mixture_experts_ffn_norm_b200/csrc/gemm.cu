@@ -153,12 +153,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
     __shared__ __align__(8) uint64_t tfull_bar[2];
     __shared__ __align__(8) uint64_t tempty_bar[2];
     __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ __align__(8) uint64_t xchg_bar;        // FP8 up: row maxima exchanged between the warpgroups
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
     __shared__ int ts_sh[kMaxExperts + 2];
     __shared__ int rb_sh[kMaxExperts + 1];
     __shared__ int rc_sh[kMaxExperts + 1];
-    __shared__ float amax_sh[2][kBM];
+    __shared__ float amax_sh[2][2][kBM];             // [tile parity][warpgroup][row]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr bool kAct8 = kFp8 && !kA16;               // FP8 activations, FP8 MMAs
@@ -194,6 +195,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
             mbar_init(&tempty_bar[b], 8);
         }
         mbar_init(&drain_bar, 1);
+        mbar_init(&xchg_bar, 256);
         abort_sh = 0;
         fence_barrier_init();
     }
@@ -367,7 +369,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
         uint8_t* ostage = smem + NS * SB + (warp - 4) * kOutStageBytes;
         const uint32_t tl = tmem + (static_cast<uint32_t>(q * 32) << 16);
         int abuf = 0;
-        uint32_t aphase = 0;
+        uint32_t aphase = 0, xpar = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
             Tile ti;
             decode_tile(t, ts_sh, rb_sh, rc_sh, p, kMode, ti);
@@ -487,10 +489,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tm_a_r, const __grid_constant__ 
                         accf[j] = silu_mul(accf[j], accf[64 + j]);
                         amax = fmaxf(amax, fabsf(accf[j]));
                     }
-                    amax_sh[c][r] = amax;
-                    named_bar_sync(1, 256);
-                    amax = fmaxf(amax, amax_sh[c ^ 1][r]);
-                    named_bar_sync(1, 256);
+                    // the row's other 64 columns belong to the other warpgroup: exchange the maxima through
+                    // shared memory, double-buffered by tile, behind a bounded wait (a hardware barrier
+                    // would wait forever for a warp that left after a timeout elsewhere)
+                    amax_sh[xpar][c][r] = amax;
+                    mbar_arrive(&xchg_bar);
+                    mbar_spin(&xchg_bar, xpar, &abort_sh, p.status, 0x32);
+                    amax = fmaxf(amax, amax_sh[xpar][c ^ 1][r]);
+                    xpar ^= 1u;
                     const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
                     const float rsc = __frcp_rn(sc);
                     // the row's 64 e4m3 codes -> this warp's staging rows -> one TMA store of 32 x 64 bytes

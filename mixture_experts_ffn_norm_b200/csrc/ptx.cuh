@@ -267,11 +267,6 @@ __device__ __forceinline__ void regs_inc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// Named barrier among `nthreads` threads (ids 1..15; 0 is __syncthreads).
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // error-free sum of two doubles: (s, e) with s + e == a + b exactly (TwoSum)
 __device__ __forceinline__ void two_sum(double a, double b, double& s, double& e) {
     s = __dadd_rn(a, b);
