@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -36,6 +37,60 @@ EncodeTiledFn get_encode() {
     return fn;
 }
 
+// Host-side cache of encoded tensor maps.  A map is a pure function of its arguments (address,
+// type, extents, strides, box, swizzle), so the key is all of them and an entry never goes stale;
+// a forward call then encodes only maps it has not seen.  Bounded: cleared when it grows large.
+struct MapKey {
+    const void* base;
+    uint64_t d0, d1, stride;
+    uint32_t b0, b1;
+    int dtype, swizzle, promo;
+    bool operator==(const MapKey& o) const {
+        return base == o.base && d0 == o.d0 && d1 == o.d1 && stride == o.stride && b0 == o.b0 && b1 == o.b1 &&
+               dtype == o.dtype && swizzle == o.swizzle && promo == o.promo;
+    }
+};
+struct MapKeyHash {
+    size_t operator()(const MapKey& k) const {
+        uint64_t h = reinterpret_cast<uintptr_t>(k.base);
+        for (uint64_t v : {k.d0, k.d1, k.stride, static_cast<uint64_t>(k.b0) << 32 | k.b1,
+                           static_cast<uint64_t>(k.dtype) << 16 | static_cast<uint64_t>(k.swizzle) << 8 |
+                               static_cast<uint64_t>(k.promo)})
+            h = (h ^ v) * 0x100000001B3ull;
+        return static_cast<size_t>(h ^ (h >> 29));
+    }
+};
+
+bool encode_cached(CUtensorMap* map, CUtensorMapDataType dtype, void* base, uint64_t d0, uint64_t d1,
+                   uint64_t stride, uint32_t b0, uint32_t b1, CUtensorMapSwizzle swizzle,
+                   CUtensorMapL2promotion promo) {
+    static std::mutex mu;
+    static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+    const MapKey key{base, d0, d1, stride, b0, b1, static_cast<int>(dtype), static_cast<int>(swizzle),
+                     static_cast<int>(promo)};
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find(key);
+        if (it != cache.end()) {
+            *map = it->second;
+            return true;
+        }
+    }
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {d0, d1};
+    const cuuint64_t strides[1] = {stride};
+    const cuuint32_t box[2] = {b0, b1};
+    const cuuint32_t estr[2] = {1u, 1u};
+    if (enc(map, dtype, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promo,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache.size() >= 4096) cache.clear();
+    cache.emplace(key, *map);
+    return true;
+}
+
 }  // namespace
 
 int num_sms() {
@@ -47,41 +102,21 @@ int num_sms() {
 // 2-D map over a row-major [rows, inner] tensor of 1-byte (fp8) or 2-byte (bf16) elements; box =
 // 128 bytes x 128 rows, 128-byte swizzle, out-of-range rows read as zero.
 bool encode_map_2d(CUtensorMap* map, const void* base, bool fp8, uint64_t inner, uint64_t rows) {
-    EncodeTiledFn enc = get_encode();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {inner, rows};
-    const cuuint64_t strides[1] = {inner * (fp8 ? 1u : 2u)};
-    const cuuint32_t box[2] = {fp8 ? 128u : 64u, 128u};
-    const cuuint32_t estr[2] = {1u, 1u};
-    return enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
-               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_cached(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                         const_cast<void*>(base), inner, rows, inner * (fp8 ? 1u : 2u), fp8 ? 128u : 64u, 128u,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 bool encode_raw_map_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows) {
-    EncodeTiledFn enc = get_encode();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {inner, rows};
-    const cuuint64_t strides[1] = {inner};
-    const cuuint32_t box[2] = {64u, 128u};
-    const cuuint32_t estr[2] = {1u, 1u};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_cached(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, const_cast<void*>(base), inner, rows, inner, 64u, 128u,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 bool encode_store_map_2d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t inner, uint64_t rows,
                          uint32_t box_inner) {
-    EncodeTiledFn enc = get_encode();
-    if (!enc) return false;
-    const cuuint64_t dims[2] = {inner, rows};
-    const cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elem_bytes)};
-    const cuuint32_t box[2] = {box_inner, 32u};
-    const cuuint32_t estr[2] = {1u, 1u};
-    return enc(map, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return encode_cached(map, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                         const_cast<void*>(base), inner, rows, inner * static_cast<uint64_t>(elem_bytes), box_inner,
+                         32u, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE);
 }
 
 bool make_layout(const moe_config_t& c, Layout& L) {
