@@ -145,6 +145,32 @@ moe_status_t moe_forward_next_norm(const moe_config_t* cfg, const void* x, const
                                    void* next_xn, void* next_residual, void* workspace,
                                    size_t workspace_bytes, void* stream);
 
+/* One rank's share of the expert-parallel layer ("MoE update" page, MoE.forward excerpt: a rank
+ * runs the experts in [experts_start_idx, experts_end_idx) on the tokens routed to them and adds
+ * their weighted outputs into a float32 y, `dist.all_reduce(y)` sums the ranks, the shared
+ * expert is added and the result is cast to x's dtype).  Every rank computes the same ffn_norm and
+ * routing over all E experts; the GEMMs run only experts [expert_begin, expert_end) (and the
+ * shared expert when with_shared != 0, on exactly one rank).
+ *   y_partial     [T, d] float32         sum over the token's slots routed to this rank's experts
+ *                                        of weight * expert output (+ the shared output), not
+ *                                        rounded; the caller sums the ranks' partials and casts
+ *                                        once to bf16 (see expert_parallel_forward in the binding)
+ *   w             routed weights of this rank's experts must be valid at their places in the
+ *                 stacked [E, ...] layout; the others are not read
+ *   residual_out  as moe_forward
+ * 0 <= expert_begin <= expert_end <= E.  MOE_ERR_UNSUPPORTED for a dense block.  Other arguments,
+ * errors and ownership as moe_forward. */
+moe_status_t moe_forward_expert_slice(const moe_config_t* cfg, const void* x, const void* residual,
+                                      const float* norm_w, const void* gate_w, const float* gate_bias,
+                                      const moe_weights_t* w, int32_t expert_begin, int32_t expert_end,
+                                      int32_t with_shared, float* y_partial, void* residual_out,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* out[i] = bf16(y[i]) (round to nearest even) for n float32 values, n a multiple of 4; y 16-byte
+ * and out 8-byte aligned.  The final cast of the expert-parallel layer after the ranks' partial
+ * sums are reduced (the pages' `y.type_as(x)`). */
+moe_status_t moe_round_bf16(const float* y, void* out, int64_t n, void* stream);
+
 /* moe_forward that also records caller-created CUDA events (cudaEvent_t passed as void*) on
  * `stream` at the stage boundaries, for timing individual kernels inside a running workload:
  *   events[0] before the first launch      events[4] after the permutation kernels

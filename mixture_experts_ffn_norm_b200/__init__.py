@@ -19,7 +19,8 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
 MOE_W_BF16, MOE_W_FP8_E4M3_B128 = 0, 1
 MOE_ACT_FP8_1x128, MOE_ACT_BF16 = 0, 1
 
-EXPORTS = ("moe_workspace_bytes", "moe_forward", "moe_forward_traced", "moe_forward_next_norm", "moe_get_status",
+EXPORTS = ("moe_workspace_bytes", "moe_forward", "moe_forward_traced", "moe_forward_next_norm",
+           "moe_forward_expert_slice", "moe_round_bf16", "moe_get_status",
            "moe_debug_routing",
            "moe_debug_norm", "moe_route_noalloc", "moe_selftest_wait_timeout", "moe_launches_per_forward",
            "moe_status_string")
@@ -62,6 +63,11 @@ def lib() -> C.CDLL:
         L.moe_forward_next_norm.restype = C.c_int
         L.moe_forward_next_norm.argtypes = [cfgp, vp, vp, vp, vp, vp, C.POINTER(moe_weights_t), vp, vp, vp, vp, vp,
                                             C.c_size_t, vp]
+        L.moe_forward_expert_slice.restype = C.c_int
+        L.moe_forward_expert_slice.argtypes = [cfgp, vp, vp, vp, vp, vp, C.POINTER(moe_weights_t), C.c_int32, C.c_int32,
+                                               C.c_int32, vp, vp, vp, C.c_size_t, vp]
+        L.moe_round_bf16.restype = C.c_int
+        L.moe_round_bf16.argtypes = [vp, vp, C.c_int64, vp]
         L.moe_get_status.restype = C.c_int
         L.moe_get_status.argtypes = [vp, vp]
         L.moe_debug_routing.restype = C.c_int
@@ -170,6 +176,53 @@ def moe_forward_next_norm(cfg: Config, x, residual, norm_w, gate_w, gate_bias, w
     if check and rc != MOE_OK:
         raise MoeError(rc, "moe_forward_next_norm")
     return rc
+
+
+def moe_forward_expert_slice(cfg: Config, x, residual, norm_w, gate_w, gate_bias, weights, expert_begin, expert_end,
+                             with_shared, y_partial, residual_out, workspace, stream=None, check=True) -> int:
+    """One rank's float32 partial of the expert-parallel layer (see include/moe.h)."""
+    ws = weights if isinstance(weights, moe_weights_t) else weights_struct(weights)
+    rc = lib().moe_forward_expert_slice(C.byref(cfg.c()), _ptr(x), _ptr(residual), _ptr(norm_w), _ptr(gate_w),
+                                        _ptr(gate_bias), C.byref(ws), int(expert_begin), int(expert_end),
+                                        int(bool(with_shared)), _ptr(y_partial), _ptr(residual_out), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream))
+    if check and rc != MOE_OK:
+        raise MoeError(rc, "moe_forward_expert_slice")
+    return rc
+
+
+def moe_round_bf16(y, out, stream=None, check=True) -> int:
+    rc = lib().moe_round_bf16(_ptr(y), _ptr(out), y.numel(), _stream(stream))
+    if check and rc != MOE_OK:
+        raise MoeError(rc, "moe_round_bf16")
+    return rc
+
+
+def expert_parallel_forward(layer: "MoELayer", x, residual, out, residual_out, rank: int, world: int, group=None,
+                            stream=None):
+    """The expert-parallel layer on one rank ("MoE update" page, MoE.forward excerpt): this rank runs
+    the contiguous expert range [rank * E / world, (rank + 1) * E / world) (rank 0 also the shared
+    expert) into a float32 partial, the partials are summed over the ranks with
+    torch.distributed.all_reduce (NCCL for device tensors; a CPU-only backend such as gloo sums a
+    host copy), and the sum is rounded once to bf16 into ``out``.  Every rank gets the full output."""
+    import torch
+    import torch.distributed as dist
+    cfg, t = layer.cfg, layer.t
+    E = cfg.n_experts
+    if E % world:
+        raise ValueError("n_experts must divide evenly over the ranks")
+    per = E // world
+    y = torch.empty(cfg.num_tokens, cfg.dim, dtype=torch.float32, device=x.device)
+    moe_forward_expert_slice(cfg, x, residual, t["norm_w"], t["gate_w"], t.get("gate_bias"), layer.wstruct,
+                             rank * per, (rank + 1) * per, rank == 0, y, residual_out, layer.workspace, stream)
+    if dist.get_backend(group) == "nccl":
+        dist.all_reduce(y, group=group)
+    else:
+        host = y.cpu()
+        dist.all_reduce(host, group=group)
+        y.copy_(host)
+    moe_round_bf16(y, out, stream)
+    return out
 
 
 def moe_get_status(workspace, stream=None) -> int:

@@ -285,17 +285,24 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
                                  const float* norm_w, const void* gate_w, const float* gate_bias,
                                  const moe_weights_t* w, void* out, void* residual_out, void* workspace,
                                  size_t workspace_bytes, void* stream_, void* const* events, int n_events,
-                                 const float* next_norm_w = nullptr, void* next_xn = nullptr) {
+                                 const float* next_norm_w = nullptr, void* next_xn = nullptr,
+                                 float* y_partial = nullptr, int ebeg = 0, int eend = -1, bool shared_here = true) {
     Layout L;
     moe_status_t st = check_config(cfg, L);
     if (st != MOE_OK) return st;
+    const bool slice = y_partial != nullptr;   // expert slice: float32 partial of experts [ebeg, eend)
+    if (eend < 0) eend = L.E;
+    if (slice && (L.dense || next_xn)) return MOE_ERR_UNSUPPORTED;
+    if (slice && (ebeg < 0 || ebeg > eend || eend > L.E || !aligned16(y_partial) || y_partial == x ||
+                  y_partial == residual || y_partial == residual_out))
+        return MOE_ERR_INVALID_ARG;
     const bool next = next_xn != nullptr;   // the next block's attn_norm fused into the combine
     if (next && L.dense) return MOE_ERR_UNSUPPORTED;
     if (next && (!next_norm_w || !residual || !residual_out)) return MOE_ERR_INVALID_ARG;
     if (next && (next_xn == x || next_xn == residual || next_xn == out || next_xn == residual_out ||
                  !aligned16(next_xn) || !aligned16(next_norm_w)))
         return MOE_ERR_INVALID_ARG;
-    if (!x || !norm_w || !w || (!out && !next)) return MOE_ERR_INVALID_ARG;
+    if (!x || !norm_w || !w || (!out && !next && !slice)) return MOE_ERR_INVALID_ARG;
     if (residual && !residual_out) return MOE_ERR_INVALID_ARG;
     if (!L.dense) {
         if (!gate_w || !w->w1 || !w->w3 || !w->w2) return MOE_ERR_INVALID_ARG;
@@ -377,7 +384,7 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
 
     // 4. permutation by expert
     const int ntu_r = L.I / 128, ntu_s = L.Is / 128, ntd = L.d / 256;
-    MOE_TRY(launch_route(L, ntu_r, ntu_s, ntd, ntd, ws, s));
+    MOE_TRY(launch_route(L, ntu_r, ntu_s, ntd, ntd, ws, s, ebeg, eend, shared_here));
     MOE_TRY(mark(4));
 
     const int G = L.E + (L.Is > 0 ? 1 : 0);
@@ -489,7 +496,9 @@ static moe_status_t forward_impl(const moe_config_t* cfg, const void* x, const v
     }
     MOE_TRY(mark(6));
     // 7. weighted combine + shared add -> out
-    if (next)
+    if (slice)
+        MOE_TRY(launch_combine_partial(L, y_partial, ebeg, eend, shared_here, ws, s));
+    else if (next)
         MOE_TRY(launch_combine_next_norm(L, out, next_norm_w, cfg->eps, residual_out, next_xn, ws, s));
     else
         MOE_TRY(launch_combine(L, out, ws, s));
@@ -513,6 +522,25 @@ extern "C" moe_status_t moe_forward_next_norm(const moe_config_t* cfg, const voi
     if (!next_xn) return MOE_ERR_INVALID_ARG;
     return forward_impl(cfg, x, residual, norm_w, gate_w, gate_bias, w, out, next_residual, workspace,
                         workspace_bytes, stream, nullptr, 0, next_norm_w, next_xn);
+}
+
+extern "C" moe_status_t moe_forward_expert_slice(const moe_config_t* cfg, const void* x, const void* residual,
+                                                 const float* norm_w, const void* gate_w, const float* gate_bias,
+                                                 const moe_weights_t* w, int32_t expert_begin, int32_t expert_end,
+                                                 int32_t with_shared, float* y_partial, void* residual_out,
+                                                 void* workspace, size_t workspace_bytes, void* stream) {
+    if (!y_partial) return MOE_ERR_INVALID_ARG;
+    return forward_impl(cfg, x, residual, norm_w, gate_w, gate_bias, w, nullptr, residual_out, workspace,
+                        workspace_bytes, stream, nullptr, 0, nullptr, nullptr, y_partial, expert_begin, expert_end,
+                        with_shared != 0);
+}
+
+extern "C" moe_status_t moe_round_bf16(const float* y, void* out, int64_t n, void* stream) {
+    if (!y || !out || n < 0 || (n & 3) || !aligned16(y) || (reinterpret_cast<uintptr_t>(out) & 7u))
+        return MOE_ERR_INVALID_ARG;
+    if (n == 0) return MOE_OK;
+    MOE_TRY(launch_round_bf16(y, out, n, static_cast<cudaStream_t>(stream)));
+    return MOE_OK;
 }
 
 extern "C" moe_status_t moe_forward_traced(const moe_config_t* cfg, const void* x, const void* residual,

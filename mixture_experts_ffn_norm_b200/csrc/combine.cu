@@ -178,7 +178,76 @@ combine_next_norm_kernel(const uint4* __restrict__ y, const uint4* __restrict__ 
     }
 }
 
+// Expert slice (the pages' expert-parallel MoE.forward: each rank adds the outputs of its own
+// experts into a float32 y, then `dist.all_reduce(y)`): the token's slots routed to experts in
+// [ebeg, eend), weighted, in slot order, plus the shared expert's row when it ran on this rank;
+// float32 out, no rounding (the sum over ranks is rounded once after the reduction).
+__global__ void __launch_bounds__(kCombineThreads)
+combine_partial_kernel(const uint4* __restrict__ y, const uint4* __restrict__ ysh, const int* __restrict__ row_of,
+                       const int* __restrict__ idx, const float* __restrict__ w, int nv, int k, int ebeg, int eend,
+                       float4* __restrict__ out) {
+    __shared__ int rows[kMaxExperts];
+    __shared__ float ws[kMaxExperts];
+    const int t = blockIdx.x;
+    for (int j = threadIdx.x; j < k; j += kCombineThreads) {
+        const int e = idx[static_cast<size_t>(t) * k + j];
+        rows[j] = row_of[static_cast<size_t>(t) * k + j];
+        ws[j] = (e >= ebeg && e < eend) ? w[static_cast<size_t>(t) * k + j] : 0.0f;   // 0: not this rank's
+    }
+    __syncthreads();
+    const int per = (nv + gridDim.y - 1) / gridDim.y;
+    const int v0 = blockIdx.y * per, v1 = min(nv, v0 + per);
+    for (int v = v0 + threadIdx.x; v < v1; v += kCombineThreads) {
+        float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < k; ++j)
+            if (ws[j] != 0.0f) add_bf16x8(a, y[static_cast<size_t>(rows[j]) * nv + v], ws[j]);
+        if (ysh) {
+            const uint4 sh = ysh[static_cast<size_t>(t) * nv + v];
+            const uint32_t u[4] = {sh.x, sh.y, sh.z, sh.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                a[2 * e] += __uint_as_float(u[e] << 16);
+                a[2 * e + 1] += __uint_as_float(u[e] & 0xFFFF0000u);
+            }
+        }
+        float4* o = out + (static_cast<size_t>(t) * nv + v) * 2;
+        o[0] = make_float4(a[0], a[1], a[2], a[3]);
+        o[1] = make_float4(a[4], a[5], a[6], a[7]);
+    }
+}
+
 }  // namespace
+
+namespace {
+// y [n] float32 -> bf16, round to nearest even (the layer's output cast, `y.type_as(x)`)
+__global__ void round_bf16_kernel(const float4* __restrict__ y, uint2* __restrict__ out, int64_t n4) {
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float4 v = y[i];
+        out[i] = make_uint2(pack2(v.x, v.y), pack2(v.z, v.w));
+    }
+}
+}  // namespace
+
+cudaError_t launch_round_bf16(const float* y, void* out, int64_t n, cudaStream_t s) {
+    const int64_t n4 = n / 4;
+    const int grid = static_cast<int>(std::min<int64_t>((n4 + 255) / 256, 8 * num_sms()));
+    round_bf16_kernel<<<std::max(grid, 1), 256, 0, s>>>(reinterpret_cast<const float4*>(y), static_cast<uint2*>(out), n4);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine_partial(const Layout& L, float* y_partial, int ebeg, int eend, bool shared_here,
+                                   uint8_t* ws, cudaStream_t s) {
+    const int nv = L.d / 8;
+    int parts = (4 * num_sms() + L.T - 1) / L.T;
+    parts = std::max(1, std::min({parts, 8, nv / kCombineThreads}));
+    combine_partial_kernel<<<dim3(L.T, parts), kCombineThreads, 0, s>>>(
+        reinterpret_cast<const uint4*>(ws + L.y),
+        (L.Is > 0 && shared_here) ? reinterpret_cast<const uint4*>(ws + L.y_sh) : nullptr,
+        reinterpret_cast<const int*>(ws + L.row_of), reinterpret_cast<const int*>(ws + L.idx),
+        reinterpret_cast<const float*>(ws + L.w), nv, L.k, ebeg, eend, reinterpret_cast<float4*>(y_partial));
+    return cudaGetLastError();
+}
 
 cudaError_t launch_combine_next_norm(const Layout& L, void* out, const float* gain, float eps, void* resid,
                                      void* xn_next, uint8_t* ws, cudaStream_t s) {

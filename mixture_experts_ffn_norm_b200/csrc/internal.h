@@ -87,8 +87,13 @@ cudaError_t launch_gemm(int mode, bool fp8, bool a16, const TensorMaps& maps, co
                         cudaStream_t s);
 cudaError_t launch_topk(const Layout& L, const void* gate_w, const float* gate_bias, uint8_t* ws, cudaStream_t s);
 cudaError_t launch_route(const Layout& L, int ntu_r, int ntu_s, int ntd_r, int ntd_s, uint8_t* ws,
-                         cudaStream_t s);
+                         cudaStream_t s, int ebeg, int eend, bool shared_here);
 cudaError_t launch_combine(const Layout& L, void* out, uint8_t* ws, cudaStream_t s);
+// expert slice: y_partial [T, d] float32 = sum over the token's slots routed to experts in
+// [ebeg, eend) of w * y (+ the shared expert's row when it ran here); no rounding
+cudaError_t launch_round_bf16(const float* y, void* out, int64_t n, cudaStream_t s);
+cudaError_t launch_combine_partial(const Layout& L, float* y_partial, int ebeg, int eend, bool shared_here,
+                                   uint8_t* ws, cudaStream_t s);
 // the combine with the next block's RMSNorm: resid holds the block's new residual on entry and the
 // next residual on exit; out (the MoE update) may be NULL
 cudaError_t launch_combine_next_norm(const Layout& L, void* out, const float* gain, float eps, void* resid,

@@ -58,7 +58,8 @@ __device__ int block_exclusive_scan(int v, int* sh, int* total) {
 __global__ void __launch_bounds__(kRouteThreads)
 scan_kernel(int* __restrict__ chunk_hist, int nchunks, int E, int T, int has_shared, int ntu_r, int ntu_s,
             int ntd_r, int ntd_s, int* __restrict__ counts, int* __restrict__ offsets, int* __restrict__ row_base,
-            int* __restrict__ row_count, int* __restrict__ ts_up, int* __restrict__ ts_down) {
+            int* __restrict__ row_count, int* __restrict__ ts_up, int* __restrict__ ts_down, int ebeg, int eend,
+            int shared_here) {
     __shared__ int sh[kRouteThreads];
     const int e = threadIdx.x;
     int cnt = 0;
@@ -70,10 +71,12 @@ scan_kernel(int* __restrict__ chunk_hist, int nchunks, int E, int T, int has_sha
         }
     }
     const int mtiles = (cnt + kBM - 1) / kBM;
+    // every expert keeps its rows; only the experts in [ebeg, eend) get GEMM tiles (an expert slice)
+    const int mine = (e >= ebeg && e < eend) ? mtiles : 0;
     int tot_rows, tot_up, tot_down;
     const int off = block_exclusive_scan(mtiles * kBM, sh, &tot_rows);
-    const int tu = block_exclusive_scan(mtiles * ntu_r, sh, &tot_up);
-    const int td = block_exclusive_scan(mtiles * ntd_r, sh, &tot_down);
+    const int tu = block_exclusive_scan(mine * ntu_r, sh, &tot_up);
+    const int td = block_exclusive_scan(mine * ntd_r, sh, &tot_down);
     if (e < E) {
         counts[e] = cnt;
         offsets[e] = off;
@@ -90,8 +93,8 @@ scan_kernel(int* __restrict__ chunk_hist, int nchunks, int E, int T, int has_sha
             const int mt = (T + kBM - 1) / kBM;
             row_base[E] = 0;
             row_count[E] = T;
-            ts_up[E + 1] = tot_up + mt * ntu_s;
-            ts_down[E + 1] = tot_down + mt * ntd_s;
+            ts_up[E + 1] = tot_up + (shared_here ? mt * ntu_s : 0);
+            ts_down[E + 1] = tot_down + (shared_here ? mt * ntd_s : 0);
         }
     }
 }
@@ -170,7 +173,8 @@ gather_kernel(const int* __restrict__ row_of, int T, int k, const uint4* __restr
 
 }  // namespace
 
-cudaError_t launch_route(const Layout& L, int ntu_r, int ntu_s, int ntd_r, int ntd_s, uint8_t* ws, cudaStream_t s) {
+cudaError_t launch_route(const Layout& L, int ntu_r, int ntu_s, int ntd_r, int ntd_s, uint8_t* ws, cudaStream_t s,
+                         int ebeg, int eend, bool shared_here) {
     const int N = L.T * L.k;
     int* idx = reinterpret_cast<int*>(ws + L.idx);
     int* chunk = reinterpret_cast<int*>(ws + L.chunk_hist);
@@ -180,7 +184,7 @@ cudaError_t launch_route(const Layout& L, int ntu_r, int ntu_s, int ntd_r, int n
                                             reinterpret_cast<int*>(ws + L.counts), reinterpret_cast<int*>(ws + L.offsets),
                                             reinterpret_cast<int*>(ws + L.row_base),
                                             reinterpret_cast<int*>(ws + L.row_count), reinterpret_cast<int*>(ws + L.ts_up),
-                                            reinterpret_cast<int*>(ws + L.ts_down));
+                                            reinterpret_cast<int*>(ws + L.ts_down), ebeg, eend, shared_here ? 1 : 0);
     scatter_kernel<<<L.nchunks, kRouteThreads, 0, s>>>(idx, N, L.E, L.k, chunk, reinterpret_cast<int*>(ws + L.offsets),
                                                        reinterpret_cast<int*>(ws + L.row_of),
                                                        reinterpret_cast<int*>(ws + L.row_token));
@@ -262,7 +266,7 @@ extern "C" moe_status_t moe_route_noalloc(const int32_t* idx, int32_t num_tokens
     if (cudaMemsetAsync(row_token, 0xFF, static_cast<size_t>(rows) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
     hist_kernel<<<nchunks, kRouteThreads, 0, s>>>(idx, N, E, hist, nullptr);
     scan_kernel<<<1, kRouteThreads, 0, s>>>(hist, nchunks, E, num_tokens, 0, 1, 1, 1, 1, counts, offsets, row_base,
-                                            row_count, ts_up, ts_down);
+                                            row_count, ts_up, ts_down, 0, E, 0);
     scatter_kernel<<<nchunks, kRouteThreads, 0, s>>>(idx, N, E, top_k, hist, offsets, row_of, row_token);
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -22,7 +22,7 @@ def _built():
 def declared_functions():
     src = open(os.path.join(ROOT, "include", "moe.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(moe_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_every_declared_symbol_is_exported():
@@ -88,3 +88,22 @@ def test_forward_rejects_bad_arguments_without_touching_the_device():
     dense = moe.Config(64, 256, 128, 0, 0, 256, moe.MOE_W_BF16, moe.MOE_ACT_BF16).c()
     assert nn(cfg=dense) == moe.MOE_ERR_UNSUPPORTED
     assert moe.status_string(moe.MOE_ERR_WORKSPACE) == "workspace missing or too small"
+
+
+def test_expert_slice_and_round_reject_bad_arguments_without_touching_the_device():
+    L = moe.lib()
+    cfg = moe.Config.from_shape(synthetic.CONFIGS["C1"]).c()
+    fake = 1 << 20
+    w = moe.moe_weights_t(fake, fake, fake, None, None, None, fake, fake, fake, None, None, None)
+    need = L.moe_workspace_bytes(C.byref(cfg))
+    sl = lambda cfg=cfg, b=0, e=4, y=fake + 65536: L.moe_forward_expert_slice(
+        C.byref(cfg), fake, fake, fake, fake, None, C.byref(w), b, e, 1, y, fake + 8192, fake, need, None)
+    assert sl(y=None) == moe.MOE_ERR_INVALID_ARG
+    assert sl(b=5, e=4) == moe.MOE_ERR_INVALID_ARG            # empty range reversed
+    assert sl(e=9) == moe.MOE_ERR_INVALID_ARG                  # beyond E = 8
+    assert sl(y=fake) == moe.MOE_ERR_INVALID_ARG               # aliases x
+    dense = moe.Config(64, 256, 128, 0, 0, 256, moe.MOE_W_BF16, moe.MOE_ACT_BF16).c()
+    assert sl(cfg=dense) == moe.MOE_ERR_UNSUPPORTED
+    assert L.moe_round_bf16(fake, fake + 4096, 6, None) == moe.MOE_ERR_INVALID_ARG   # not a multiple of 4
+    assert L.moe_round_bf16(None, fake, 8, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_round_bf16(fake, fake, 0, None) == moe.MOE_OK
