@@ -1,10 +1,11 @@
 """Parity of the CUDA path (through the C ABI) with the CPU oracle on the same seeded inputs.
 
-Small and ragged layers are compared on every token; the full-size workloads (decode, prefill,
-skewed routing) are run exactly as bench.py launches them and compared on a seeded token sample
-that covers every expert the GPU used, with routing checked on all tokens.  The five workloads
-use the stated output bound max|err| <= 2e-2 * RMS as is; the extra structural layers also
-accept a one-bf16-step difference per element (see harness.check_out).
+Small and ragged layers and the decode workload are compared on every token; the other full-size
+workloads (mid-size, prefill, skewed routing) are run exactly as bench.py launches them and
+compared on a seeded token sample that covers every expert the GPU used, with routing checked on
+all tokens.  The five workloads use the stated output bound max|err| <= 2e-2 * RMS as is; the
+extra structural layers also accept a one-bf16-step difference per element (see
+harness.check_out).
 """
 import dataclasses
 import json
@@ -147,7 +148,8 @@ def test_full_size_workloads(name, n_sample):
     allt = np.arange(shape.T, dtype=np.int32)
     check_norm(run, route, allt, report)
     check_routing(run, route, allt, report)
-    toks = sample_tokens(run, route, n_sample, seed=shape.seed)
+    # the decode workload is compared on every token; the larger ones on a sample
+    toks = allt if name == "C3" else sample_tokens(run, route, n_sample, seed=shape.seed)
     ref = o.forward(toks)
     check_out(run, ref, toks, report)
     report["sampled_tokens"] = int(len(toks))
