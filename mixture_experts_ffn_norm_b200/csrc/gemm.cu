@@ -13,13 +13,17 @@
 // scaling does not apply.  Each 128-wide K block is therefore accumulated into its own TMEM buffer
 // and promoted by the epilogue warps: acc += P_kb * (s_act[row, kb] * s_w[nblk, kb]) in float32
 // registers.  Two TMEM buffers (2 x 256 columns) let the MMA of block kb+1 run while block kb is
-// promoted.  bf16 operands simply accumulate the whole K in TMEM.
+// promoted.  bf16 operands simply accumulate the whole K in TMEM.  With FP8 weights and bf16
+// activations (kA16) each stage's e4m3 weight tile is widened to bf16 in shared memory, the MMAs
+// are bf16 and every 128-wide K block (two 64-wide stages) is promoted with its weight scale.
+// The router-logits launch may split K into parts that write float32 partial tiles (few tokens).
 //
 // Warp roles (384 threads = 3 warpgroups, one CTA per SM, persistent over a device-side tile table):
 //   warp 0      issues the TMA loads of A (128 x 128 B) and B (256 x 128 B) per stage (one elected lane)
 //   warp 1      issues tcgen05.mma (M=128, N=256, K=32 bytes per instruction): the whole warp runs the
 //               loop and waits, one elected lane issues
-//   warps 2-3   idle (they only hand their registers back)
+//   warps 2-3   kA16: widen the stage's e4m3 weight tile to bf16; otherwise idle (they only hand
+//               their registers back)
 //   warps 4..11 epilogue: warp w reads TMEM lanes 32*(w%4).., column half (w-4)/4
 // Each promotion reads 64 TMEM columns per tcgen05.ld (two per K block per thread).
 // The MMA thread and the epilogue poll their barriers (mbar_spin) rather than suspend in try_wait:
