@@ -2,8 +2,13 @@
 // sequence of one forward pass.  Nothing here waits on the device except moe_get_status.
 //
 // Launch sequence (one stream, no host sync; every routing-dependent size is read on the device):
-//   norm -> gate GEMM (logits) -> top-k with float64 re-decision -> hist -> scan -> scatter
-//   -> gather -> grouped GEMM up (w1|w3 + SwiGLU) -> grouped GEMM down (w2) -> combine
+//   norm -> gate GEMM (logits; K split over CTAs for few tokens) -> top-k (float32 pass, then the
+//   float64 re-decision of the listed near-tie tokens) -> hist -> scan -> scatter -> gather
+//   -> grouped GEMM up (w1|w3 + SwiGLU) -> grouped GEMM down (w2) -> combine
+// The combine has two variants: with the next block's RMSNorm fused in (moe_forward_next_norm)
+// and the float32 partial of an expert slice (moe_forward_expert_slice).  A dense block
+// (n_experts = 0) runs norm -> up -> down, the second GEMM writing the output.  Tensor maps are
+// cached on the host (a map is a pure function of its arguments).
 #include <algorithm>
 #include <cstring>
 #include <mutex>

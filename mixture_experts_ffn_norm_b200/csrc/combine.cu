@@ -9,6 +9,8 @@
 // float32 in slot order, adds the shared expert's row and rounds once to bf16.  A token's row is
 // split over several CTAs when there are few tokens (decode), so that every SM has loads in flight;
 // each thread issues the loads of up to 8 slots before their FMAs.
+// Also here: the same combine with the next block's RMSNorm fused in, the float32 partial of an
+// expert slice, and the final bf16 cast of the reduced partials.
 #include <cuda_bf16.h>
 
 #include <algorithm>

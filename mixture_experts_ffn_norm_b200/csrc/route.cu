@@ -9,7 +9,10 @@
 //   scatter : every entry gets its row in the permuted order (token order inside an expert,
 //             so the permutation is deterministic);
 //   gather  : the permuted activation rows (FP8 codes or bf16) and their group scales are
-//             copied next to each other so a TMA box of 128 rows is one expert's tile.
+//             copied next to each other so a TMA box of 128 rows is one expert's tile (one warp
+//             per token reads its row once and writes its k copies).
+// For an expert slice the scan gives only the experts in [ebeg, eend) GEMM tiles; every expert
+// keeps its rows in the permutation.
 #include <mutex>
 
 #include "internal.h"
