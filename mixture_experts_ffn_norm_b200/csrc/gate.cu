@@ -26,7 +26,7 @@ namespace moe {
 namespace {
 
 constexpr int kTopkWarps = 8;
-constexpr int kRedoWarps = 8;
+constexpr int kRedoWarps = 16;        // a listed token's candidates, one warp each (S rarely exceeds 16)
 constexpr int kMaxSplit = 16;          // K parts of the router-logits GEMM (the layout never makes more)
 constexpr float kCandDelta = 2e-3f;    // logit units; far above the float32 logit error
 constexpr int J = kMaxExperts / 32;    // experts per lane
@@ -303,7 +303,7 @@ cudaError_t launch_topk(const Layout& L, const void* gate_w, const float* gate_b
                                                  ws + L.flag, reinterpret_cast<int*>(ws + L.redo), status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    topk_redo_kernel<<<std::min(L.T, 2 * num_sms()), kRedoWarps * 32, 0, s>>>(
+    topk_redo_kernel<<<std::min(L.T, 4 * num_sms()), kRedoWarps * 32, 0, s>>>(
         logits, L.ksplit, gate_bias, reinterpret_cast<const uint16_t*>(ws + L.xn), static_cast<const uint16_t*>(gate_w),
         L.T, L.E, L.k, L.d, reinterpret_cast<int*>(ws + L.idx), reinterpret_cast<float*>(ws + L.w),
         reinterpret_cast<const int*>(ws + L.redo), status);
